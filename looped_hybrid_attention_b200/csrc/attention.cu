@@ -1,0 +1,303 @@
+// Full-attention execution ("Loop-9B engineering teardown" §三): GQA 16 q / 4 KV heads,
+// head dim 256, QK-norm, interleaved rotary on 0.25 of the head dims, sigmoid
+// output gate; §四: each execution writes its own KV slab.
+//
+// fa_prep_kernel : QK-norm + rotary for q (to a compact buffer) and k (into the
+//                  slab), v copied into the slab.  One warp per (token, head).
+// attn_rows_kernel: softmax attention for a block of query rows of one KV group.
+//                  One warp per (query row, q head); the Hq/Hkv heads of a group
+//                  share each K/V row through L1.  Lanes split the head dim;
+//                  scores of 8 keys are reduced together (reduce-scatter), so a
+//                  key costs ~2 shuffles.  Keys may be split across CTAs
+//                  (flash-decode); attn_combine_kernel merges the splits.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lk {
+
+// ------------------------------------------------------------------ QK-norm + rotary + KV write
+template <typename T, int DH>
+__global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, int ld_p, const T* __restrict__ q_norm,
+                                                      const T* __restrict__ k_norm, T* __restrict__ q_out,
+                                                      T* __restrict__ k_cache, T* __restrict__ v_cache, int kv_cap,
+                                                      int T_len, int pos0, int Hq, int Hkv, int rot, float base,
+                                                      float eps) {
+  constexpr int PER = DH / 32;         // contiguous elements per lane (even: rotary pairs stay local)
+  const int lane = threadIdx.x & 31;
+  const int heads = Hq + Hkv;
+  const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int b = blockIdx.y;
+  if (w >= (long)T_len * heads) return;
+  const int t = (int)(w / heads), hh = (int)(w % heads);
+  const long m = (long)b * T_len + t;
+  const int pos = pos0 + t;
+  const T* row = P + m * ld_p;
+  const bool is_q = hh < Hq;
+  const int kvh = hh - Hq;
+  const T* src = is_q ? row + hh * DH : row + 2 * Hq * DH + kvh * DH;
+  const T* gain = is_q ? q_norm : k_norm;
+  float x[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) x[u] = ldf(src + lane * PER + u);
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) ss += x[u] * x[u];
+  const float inv = rsqrtf(warp_sum(ss) / (float)DH + eps);
+#pragma unroll
+  for (int u = 0; u < PER; ++u) x[u] = x[u] * inv * ldf(gain + lane * PER + u);
+  // rotary on dims [0, rot): pair (2j, 2j+1), angle pos * base^(-2j/rot), evaluated in fp64
+#pragma unroll
+  for (int u = 0; u < PER; u += 2) {
+    const int e = lane * PER + u;
+    if (e < rot) {
+      const int j = e >> 1;
+      const double theta = pow((double)base, -2.0 * (double)j / (double)rot);
+      double ang = (double)pos * theta;
+      ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      const float c = (float)cs, s = (float)sn;
+      const float a0 = x[u], a1 = x[u + 1];
+      x[u] = a0 * c - a1 * s;
+      x[u + 1] = a0 * s + a1 * c;
+    }
+  }
+  T* dst;
+  if (is_q) {
+    dst = q_out + (m * Hq + hh) * DH;
+  } else {
+    const long slot = (((long)b * Hkv + kvh) * kv_cap + pos) * DH;
+    dst = k_cache + slot;
+    const T* vs = row + 2 * Hq * DH + Hkv * DH + kvh * DH;
+    T* vd = v_cache + slot;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) stf(dst + lane * PER + u, x[u]);
+}
+
+cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
+                    void* k_cache, void* v_cache, int kv_cap, int B, int T, int pos0, int Hq,
+                    int Hkv, int dh, int rotary_dims, float rope_base, float eps, int dtype,
+                    cudaStream_t s) {
+  if (T == 0 || B == 0) return cudaSuccess;
+  const int warps = 8;
+  dim3 grid((unsigned)(((long)T * (Hq + Hkv) + warps - 1) / warps), B);
+#define FA_PREP(TT, DHV)                                                                                   \
+  fa_prep_kernel<TT, DHV><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,               \
+                                                      (const TT*)k_norm, (TT*)q_out, (TT*)k_cache,         \
+                                                      (TT*)v_cache, kv_cap, T, pos0, Hq, Hkv, rotary_dims, \
+                                                      rope_base, eps)
+  if (dtype == BF16) {
+    if (dh == 256) FA_PREP(__nv_bfloat16, 256); else if (dh == 128) FA_PREP(__nv_bfloat16, 128);
+    else if (dh == 64) FA_PREP(__nv_bfloat16, 64); else return cudaErrorNotSupported;
+  } else {
+    if (dh == 256) FA_PREP(float, 256); else if (dh == 128) FA_PREP(float, 128);
+    else if (dh == 64) FA_PREP(float, 64); else return cudaErrorNotSupported;
+  }
+#undef FA_PREP
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ attention over rows
+// Reduce-scatter of 8 per-lane partial sums: afterwards lane L holds the full sum
+// of value index (L >> 2) & 7.
+__device__ __forceinline__ float reduce_scatter8(const float v[8], int lane) {
+  float a[4], b2[2];
+  const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float send = h4 ? v[i] : v[i + 4];
+    float keep = h4 ? v[i + 4] : v[i];
+    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float send = h3 ? a[i] : a[i + 2];
+    float keep = h3 ? a[i + 2] : a[i];
+    b2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float send = h2 ? b2[0] : b2[1];
+  float s = (h2 ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  return s;
+}
+
+template <typename T, int DH>
+__global__ void attn_rows_kernel(const T* __restrict__ q, int ld_q, const T* __restrict__ kc,
+                                 const T* __restrict__ vc, int kv_cap, const T* __restrict__ gate,
+                                 int ld_gate, T* __restrict__ out, float* __restrict__ ws, int Tq, int Tkv,
+                                 int q_off, int Hq, int Hkv, int causal, int n_split, int split_len,
+                                 float scale) {
+  constexpr int PER = DH / 32;
+  const int lane = threadIdx.x & 31, hw = threadIdx.x >> 5;    // warp = q head within the group
+  const int rep = Hq / Hkv;
+  const int t = blockIdx.x;
+  const int kvh = blockIdx.y / n_split, split = blockIdx.y % n_split;
+  const int b = blockIdx.z;
+  const int h = kvh * rep + hw;
+  const long m = (long)b * Tq + t;
+  float qq[PER], o[PER];
+  const T* qp = q + m * ld_q + (long)h * DH + lane * PER;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) { qq[u] = ldf(qp + u) * scale; o[u] = 0.f; }
+  int k_end = Tkv;
+  if (causal) k_end = min(k_end, q_off + t + 1);
+  const int k_begin = split * split_len;
+  k_end = min(k_end, k_begin + split_len);
+  const T* Kb = kc + ((long)b * Hkv + kvh) * kv_cap * DH + lane * PER;
+  const T* Vb = vc + ((long)b * Hkv + kvh) * kv_cap * DH + lane * PER;
+  float mx = -INFINITY, l = 0.f;
+  for (int p0 = k_begin; p0 < k_end; p0 += 8) {
+    float part[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      part[c] = 0.f;
+      const int p = p0 + c;
+      if (p < k_end) {
+        const T* kr = Kb + (long)p * DH;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) part[c] = fmaf(qq[u], ldf(kr + u), part[c]);
+      }
+    }
+    const float mine = reduce_scatter8(part, lane);
+    float s8[8];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      s8[c] = __shfl_sync(0xffffffffu, mine, c << 2);
+      if (p0 + c >= k_end) s8[c] = -INFINITY;
+      tmax = fmaxf(tmax, s8[c]);
+    }
+    const float mnew = fmaxf(mx, tmax);
+    const float corr = expf(mx - mnew);     // mx = -inf on the first tile -> 0
+    l *= corr;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) o[u] *= corr;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int p = p0 + c;
+      if (p < k_end) {
+        const float pc = expf(s8[c] - mnew);
+        l += pc;
+        const T* vr = Vb + (long)p * DH;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) o[u] = fmaf(pc, ldf(vr + u), o[u]);
+      }
+    }
+    mx = mnew;
+  }
+  if (n_split == 1) {
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const T* gp = gate ? gate + m * ld_gate + (long)h * DH + lane * PER : nullptr;
+    T* op = out + (m * Hq + h) * DH + lane * PER;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      float r = o[u] * inv;
+      if (gp) r *= sigmoidf_acc(ldf(gp + u));
+      stf(op + u, r);
+    }
+  } else {
+    // partials: [m, h, split] -> (max, sum, o[DH])
+    float* w = ws + ((m * Hq + h) * n_split + split) * (DH + 2);
+    if (lane == 0) { w[0] = mx; w[1] = l; }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) w[2 + lane * PER + u] = o[u];
+  }
+}
+
+template <typename T, int DH>
+__global__ void attn_combine_kernel(const float* __restrict__ ws, const T* __restrict__ gate, int ld_gate,
+                                    T* __restrict__ out, long rows, int Hq, int n_split) {
+  constexpr int PER = DH / 32;
+  const int lane = threadIdx.x & 31;
+  const long r = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // r = m * Hq + h
+  if (r >= rows) return;
+  const float* w = ws + r * n_split * (DH + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, w[s * (DH + 2)]);
+  float L = 0.f, o[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) o[u] = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float* ws_s = w + s * (DH + 2);
+    const float f = ws_s[0] == -INFINITY ? 0.f : expf(ws_s[0] - M);
+    L += f * ws_s[1];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) o[u] = fmaf(f, ws_s[2 + lane * PER + u], o[u]);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const long m = r / Hq;
+  const int h = (int)(r % Hq);
+  const T* gp = gate ? gate + m * ld_gate + (long)h * DH + lane * PER : nullptr;
+  T* op = out + r * DH + lane * PER;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    float v = o[u] * inv;
+    if (gp) v *= sigmoidf_acc(ldf(gp + u));
+    stf(op + u, v);
+  }
+}
+
+static int attn_splits(int B, int Tq, int Tkv, int Hkv) {
+  const long blocks = (long)B * Tq * Hkv;
+  int want = (int)((4L * 148 + blocks - 1) / blocks);
+  int cap = (Tkv + 511) / 512;
+  int s = want < cap ? want : cap;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : s;
+}
+
+size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
+  const int Hkv = 1;   // upper bound: splits computed with Hkv = 1 are never fewer
+  const int s = attn_splits(B, Tq, Tkv, Hkv);
+  return (size_t)B * Tq * Hq * s * (dh + 2) * sizeof(float);
+}
+
+bool gqa_supported(int dh, int Hq, int Hkv) {
+  return (dh == 64 || dh == 128 || dh == 256) && Hkv > 0 && Hq % Hkv == 0 && Hq / Hkv <= 32;
+}
+
+template <typename T, int DH>
+static cudaError_t launch_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                               const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
+                               int Hq, int Hkv, int causal, void* workspace, cudaStream_t s) {
+  int n_split = workspace ? attn_splits(B, Tq, Tkv, Hkv) : 1;
+  const int split_len = (Tkv + n_split - 1) / n_split;
+  dim3 grid(Tq, Hkv * n_split, B);
+  const int threads = 32 * (Hq / Hkv);
+  const float scale = 1.f / sqrtf((float)DH);
+  attn_rows_kernel<T, DH><<<grid, threads, 0, s>>>((const T*)q, ld_q, (const T*)k, (const T*)v, kv_cap,
+                                                   (const T*)gate, ld_gate, (T*)out, (float*)workspace, Tq,
+                                                   Tkv, q_off, Hq, Hkv, causal, n_split, split_len, scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || n_split == 1) return e;
+  const long rows = (long)B * Tq * Hq;
+  attn_combine_kernel<T, DH><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const float*)workspace, (const T*)gate,
+                                                                         ld_gate, (T*)out, rows, Hq, n_split);
+  return cudaGetLastError();
+}
+
+cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                     const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
+                     int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
+                     cudaStream_t s) {
+  if (B == 0 || Tq == 0) return cudaSuccess;
+#define ATTN(TT, DHV) \
+  return launch_attn<TT, DHV>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, workspace, s)
+  if (dtype == BF16) {
+    if (dh == 256) ATTN(__nv_bfloat16, 256);
+    if (dh == 128) ATTN(__nv_bfloat16, 128);
+    if (dh == 64) ATTN(__nv_bfloat16, 64);
+  } else {
+    if (dh == 256) ATTN(float, 256);
+    if (dh == 128) ATTN(float, 128);
+    if (dh == 64) ATTN(float, 64);
+  }
+#undef ATTN
+  return cudaErrorNotSupported;
+}
+
+}  // namespace lk

@@ -1,0 +1,58 @@
+// Internal launchers shared by the C-ABI layer and the model runtime.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lk {
+
+enum Dtype { F32 = 0, BF16 = 1 };
+enum Epilogue { EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_F32 = 3 };
+enum MhcMode { MHC_OPEN = 0, MHC_MIX = 1, MHC_ROUTE = 2, MHC_MERGE = 3 };
+
+// ldx: row stride of x in elements (0 = d); r, sum_out and y are dense [M, d].
+cudaError_t rmsnorm(const void* x, const void* r, void* sum_out, const void* w, void* y, int M,
+                    int d, float eps, int dtype, cudaStream_t s, long ldx = 0);
+cudaError_t embed(const int32_t* ids, const void* E, void* out, int M, int d, int vocab, int dtype,
+                  cudaStream_t s);
+cudaError_t argmax(const float* logits, int32_t* next, int B, int V, cudaStream_t s);
+
+cudaError_t linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
+                   void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s);
+// tcgen05 path (bf16); returns cudaErrorNotSupported for shapes it does not take.
+cudaError_t linear_tc(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
+                      void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s);
+cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, const void* R,
+                        int ldr, void* Y, int ldy, int M, int N, int K, int epi, int dtype,
+                        cudaStream_t s);
+
+cudaError_t gdn_prep(const void* P, int ld_p, const float* a_bias, const float* b_bias, void* q,
+                     void* k, void* v, float* g, float* beta, int M, int H, int dk, int dv,
+                     float eps, int dtype, cudaStream_t s);
+cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* state, void* out, int B, int T, int H, int dk,
+                      int dv, float scale, int dtype, cudaStream_t s);
+cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     float* state, void* out, int B, int H, int dk, int dv, float scale, int dtype,
+                     cudaStream_t s);
+bool gdn_supported(int dk, int dv);
+
+cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
+                    void* k_cache, void* v_cache, int kv_cap, int B, int T, int pos0, int Hq,
+                    int Hkv, int dh, int rotary_dims, float rope_base, float eps, int dtype,
+                    cudaStream_t s);
+cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                     const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
+                     int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
+                     cudaStream_t s);
+size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
+bool gqa_supported(int dh, int Hq, int Hkv);
+
+cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
+                const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,
+                int d, float eps, int iters, int dtype, cudaStream_t s);
+cudaError_t sinkhorn(const float* logits, float* out, int N, int n, int iters, cudaStream_t s);
+
+int read_and_clear_device_error();
+
+}  // namespace lk

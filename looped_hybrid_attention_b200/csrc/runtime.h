@@ -1,0 +1,56 @@
+// Model runtime: schedule, per-execution cache manager, activation workspace,
+// and the forward orchestration (prefill / hidden-state forward / decode step).
+#pragma once
+#include <string>
+#include <vector>
+
+#include "../../include/loop.h"
+#include "internal.h"
+
+struct ExecRow {
+  int exec, layer, kind, slot, in_loop;   // kind: 0 GDN, 1 full attention
+};
+
+// Execution table of a config: head layers once, the loop block `loop_passes`
+// times with shared weights, tail layers once; slots count executions per kind.
+std::vector<ExecRow> build_schedule(const loop_config& c);
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t bytes = 0;
+  ~DevBuf();
+  cudaError_t ensure(size_t want);   // grow-only
+};
+
+struct loop_model {
+  loop_config cfg;
+  std::vector<loop_layer_weights> layers;
+  const void* embed = nullptr;
+  const void* final_norm = nullptr;
+  const void* lm_head = nullptr;
+  std::vector<ExecRow> sched;
+  int n_fa = 0, n_gdn = 0;
+  int first_loop = -1, last_loop = -1;
+  size_t esize = 2;
+  // activation workspace, sized for `ws_tokens` tokens
+  long ws_tokens = 0;
+  DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, last;
+  int in_gdn = 0, in_fa = 0;
+};
+
+struct loop_cache {
+  const loop_model* model = nullptr;
+  int batch = 0, max_tokens = 0, len = 0;
+  DevBuf kv, state;
+  size_t kv_slab_elems = 0;      // elements of one K (or V) slab
+  size_t state_elems = 0;        // floats of one GDN state (all sequences)
+};
+
+// Set the thread's error message; returns `st`.
+loop_status fail(loop_status st, const std::string& msg);
+loop_status cuda_fail(cudaError_t e, const char* what);
+
+loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const void* h_in, void* h_out,
+                        float* logits_last, int B, int T, cudaStream_t s);
+loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* logits, int32_t* next,
+                       cudaStream_t s);

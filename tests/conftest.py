@@ -18,3 +18,38 @@ def golden():
     import json
     with open(os.path.join(ROOT, "tests", "golden", "pages.json")) as f:
         return json.load(f)
+
+
+# ----------------------------------------------------------------------------- shared helpers
+import numpy as np
+
+
+def rel_l2(a, b):
+    """||a - b|| / ||b|| in float64 (b is the oracle)."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
+
+
+def to64(t):
+    """Device/host tensor -> float64 numpy (exact widening)."""
+    import torch
+    t = t.detach().to("cpu")
+    if t.dtype in (torch.bfloat16, torch.float16):
+        t = t.float()
+    return t.numpy().astype(np.float64)
+
+
+# Tolerances: fp32 ops rel-L2 <= 1e-5; bf16 per-op outputs are rounded to bf16
+# (relative 2^-9 per element, so rel-L2 ~ 3e-3) -> 1e-2; bf16 end-to-end hidden
+# states 2e-2; Sinkhorn matrices 1e-6 absolute.
+TOL = {"fp32": 1e-5, "bf16": 1e-2, "bf16_e2e": 2e-2, "sinkhorn": 1e-6}
+
+
+@pytest.fixture(scope="session")
+def cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import looped_hybrid_attention_b200 as L   # noqa: F401  (fails loudly if the library is missing)
+    return torch.device("cuda:0")

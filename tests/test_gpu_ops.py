@@ -1,0 +1,412 @@
+"""Per-op parity: each C-ABI entry point on the GPU against the oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import TOL, rel_l2, to64
+from oracle import ops
+
+pytestmark = pytest.mark.gpu
+
+DT = {"fp32": torch.float32, "bf16": torch.bfloat16}
+
+
+def rnd(shape, seed, name, std=1.0, dtype="fp32", dev="cuda"):
+    return synth.normal(shape, std, seed, name).to(DT[dtype]).to(dev)
+
+
+# ----------------------------------------------------------------------------- Sinkhorn + mHC
+
+@pytest.mark.parametrize("n", [2, 3, 4])
+def test_sinkhorn_fp32(cuda, n):
+    import looped_hybrid_attention_b200 as L
+    N = 1000
+    Lg = rnd((N, n, n), 0, f"sk{n}", std=2.0)
+    out = torch.empty_like(Lg)
+    L.sinkhorn_fp32(Lg, out, 20)
+    ref = ops.sinkhorn(to64(Lg), 20)
+    assert np.abs(to64(out) - ref).max() <= TOL["sinkhorn"]
+    # zero iterations = normalised exp only
+    L.sinkhorn_fp32(Lg, out, 0)
+    e = np.exp(to64(Lg) - to64(Lg).max(axis=(1, 2), keepdims=True))
+    assert np.abs(to64(out) - e).max() < 1e-6
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19)])
+def test_mhc_modes(cuda, dtype, d, N):
+    import looped_hybrid_attention_b200 as L
+    code = L.BF16 if dtype == "bf16" else L.F32
+    eps, iters = 1e-6, 20
+    h = rnd((N, d), 1, "h", dtype=dtype)
+    F = rnd((N, d), 2, "F", dtype=dtype)
+    w_r = rnd((2 * d, 8), 3, "wr", std=0.02)
+    b_r = rnd((8,), 4, "br", std=0.5)
+    X = torch.empty((N, 2, d), dtype=DT[dtype], device=cuda)
+    x_in = torch.empty((N, d), dtype=DT[dtype], device=cuda)
+    c0 = torch.empty((N, 8), device=cuda)
+    tol = TOL[dtype]
+    # OPEN: X = (h, h), route from it
+    L.mhc_route_mix(L.MHC_OPEN, h, None, None, w_r, b_r, X, x_in, None, c0, N, d, eps, iters, code)
+    Xo = ops.mhc_open(to64(h))
+    assert np.array_equal(to64(X), Xo)
+    pre, post, res = ops.mhc_coeffs(Xo, to64(w_r), to64(b_r), eps, iters)
+    c = to64(c0)
+    assert rel_l2(c[:, 0:2], pre) < 1e-5 and rel_l2(c[:, 2:4], post) < 1e-5
+    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() < 1e-5
+    assert rel_l2(to64(x_in), ops.mhc_read(Xo, c[:, 0:2])) < tol
+    # MIX: X' = H_res X + H_post F, then route from X' as stored
+    X_prev = X.clone()
+    c1 = torch.empty_like(c0)
+    L.mhc_route_mix(L.MHC_MIX, X, F, c0, w_r, b_r, X, x_in, None, c1, N, d, eps, iters, code)
+    Xm = ops.mhc_write(to64(X_prev), to64(F), c[:, 2:4], c[:, 4:8].reshape(N, 2, 2))
+    assert rel_l2(to64(X), Xm) < tol
+    pre, post, res = ops.mhc_coeffs(to64(X), to64(w_r), to64(b_r), eps, iters)
+    c = to64(c1)
+    assert rel_l2(c[:, 0:2], pre) < 1e-5 and rel_l2(c[:, 2:4], post) < 1e-5
+    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() < 1e-5
+    assert rel_l2(to64(x_in), ops.mhc_read(to64(X), pre)) < tol
+    # ROUTE only: X unchanged
+    X_keep = X.clone()
+    L.mhc_route_mix(L.MHC_ROUTE, X, None, None, w_r, b_r, None, x_in, None, c1, N, d, eps, iters, code)
+    assert torch.equal(X, X_keep)
+    assert rel_l2(to64(c1), c) < 1e-6
+    # MERGE: mix then average the streams
+    hm = torch.empty((N, d), dtype=DT[dtype], device=cuda)
+    L.mhc_route_mix(L.MHC_MERGE, X, F, c1, None, None, None, None, hm, None, N, d, eps, iters, code)
+    Xm = ops.mhc_write(to64(X), to64(F), c[:, 2:4], c[:, 4:8].reshape(N, 2, 2))
+    assert rel_l2(to64(hm), ops.mhc_merge(Xm)) < tol
+
+
+def test_mhc_zero_routing_is_plain_residual(cuda):
+    import looped_hybrid_attention_b200 as L
+    N, d = 10, 256
+    h = rnd((N, d), 5, "h0")
+    F = rnd((N, d), 6, "F0")
+    X = torch.empty((N, 2, d), device=cuda)
+    x_in = torch.empty((N, d), device=cuda)
+    c = torch.empty((N, 8), device=cuda)
+    z = torch.zeros((2 * d, 8), device=cuda)
+    L.mhc_route_mix(L.MHC_OPEN, h, None, None, z, z[0], X, x_in, None, c, N, d, 1e-6, 20, L.F32)
+    assert torch.allclose(c, torch.tensor([0.5, 0.5, 1, 1, 0.5, 0.5, 0.5, 0.5], device=cuda))
+    assert torch.allclose(x_in, h, atol=1e-6)
+    hm = torch.empty_like(h)
+    L.mhc_route_mix(L.MHC_MERGE, X, F, c, None, None, None, None, hm, None, N, d, 1e-6, 20, L.F32)
+    assert torch.allclose(hm, h + F, atol=1e-5)
+
+
+# ----------------------------------------------------------------------------- norms, embedding, argmax
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_rmsnorm_with_residual(cuda, dtype):
+    import looped_hybrid_attention_b200 as L
+    M, d = 33, 4096
+    x, r = rnd((M, d), 7, "x", dtype=dtype), rnd((M, d), 8, "r", dtype=dtype)
+    w = rnd((d,), 9, "w", dtype=dtype, std=0.1) + 1
+    y, s = torch.empty_like(x), torch.empty_like(x)
+    L.rmsnorm(x, w, y, 1e-6)
+    assert rel_l2(to64(y), ops.rmsnorm(to64(x), to64(w), 1e-6)) < TOL[dtype]
+    L.rmsnorm(x, w, y, 1e-6, r=r, sum_out=s)
+    assert rel_l2(to64(s), to64(x) + to64(r)) < TOL[dtype]
+    assert rel_l2(to64(y), ops.rmsnorm(to64(s), to64(w), 1e-6)) < TOL[dtype]
+
+
+def test_embed_and_argmax(cuda):
+    import looped_hybrid_attention_b200 as L
+    V, d = 1000, 256
+    E = rnd((V, d), 10, "E", dtype="bf16")
+    ids = synth.uniform_ids((77,), V, 0).to(cuda)
+    out = torch.empty((77, d), dtype=torch.bfloat16, device=cuda)
+    L.embed(ids, E, out)
+    assert torch.equal(out, E[ids.long()])
+    assert L.device_error() == 0
+    bad = ids.clone()
+    bad[3] = V
+    L.embed(bad, E, out)
+    torch.cuda.synchronize()
+    assert L.device_error() == 1 and torch.all(out[3] == 0)
+    lg = rnd((5, 248320), 11, "lg")
+    lg[2, 17] = lg[2, 99] = 100.0          # tie -> lowest index
+    nx = torch.empty(5, dtype=torch.int32, device=cuda)
+    L.argmax(lg, nx)
+    ref = ops.greedy(to64(lg))
+    assert np.array_equal(nx.cpu().numpy(), ref) and nx[2].item() == 17
+
+
+# ----------------------------------------------------------------------------- projections
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("M,N,K", [(200, 300, 256), (1, 1000, 512), (130, 64, 4096)])
+def test_linear_epilogues(cuda, dtype, M, N, K):
+    import looped_hybrid_attention_b200 as L
+    X = rnd((M, K), 12, "X", dtype=dtype)
+    W = rnd((N, K), 13, "W", std=0.02, dtype=dtype)
+    W2 = rnd((N, K), 14, "W2", std=0.02, dtype=dtype)
+    R = rnd((M, N), 15, "R", dtype=dtype)
+    Y = torch.empty((M, N), dtype=DT[dtype], device=cuda)
+    ref = ops.linear(to64(X), to64(W))
+    L.linear(X, W, Y, L.EPI_STORE)
+    assert rel_l2(to64(Y), ref) < TOL[dtype]
+    L.linear(X, W, Y, L.EPI_ADD, R=R)
+    assert rel_l2(to64(Y), ref + to64(R)) < TOL[dtype]
+    L.linear(X, W, Y, L.EPI_SWIGLU, W2=W2)
+    assert rel_l2(to64(Y), ops.silu(ref) * ops.linear(to64(X), to64(W2))) < TOL[dtype]
+    Yf = torch.empty((M, N), dtype=torch.float32, device=cuda)
+    L.linear(X, W, Yf, L.EPI_F32)
+    assert rel_l2(to64(Yf), ref) < (1e-5 if dtype == "fp32" else 1e-4)
+
+
+# ----------------------------------------------------------------------------- Gated DeltaNet
+
+def _gdn_inputs(B, T, H, dk, dv, dtype, seed):
+    q = ops.l2norm(synth.normal((B, T, H, dk), 1.0, seed, "q").double().numpy(), 1e-6)
+    k = ops.l2norm(synth.normal((B, T, H, dk), 1.0, seed, "k").double().numpy(), 1e-6)
+    v = synth.normal((B, T, H, dv), 1.0, seed, "v")
+    a = synth.normal((B, T, H), 1.5, seed, "a").double().numpy()
+    b = synth.normal((B, T, H), 1.0, seed, "b").double().numpy()
+    g, beta = ops.gdn_gates(a, b, 0.0, 0.0)
+    S0 = synth.normal((B, H, dv, dk), 0.1, seed, "S0")
+    t = lambda x: torch.tensor(x).to(DT[dtype]).cuda() if not torch.is_tensor(x) else x.to(DT[dtype]).cuda()
+    return t(q), t(k), t(v), torch.tensor(g, dtype=torch.float32).cuda(), \
+        torch.tensor(beta, dtype=torch.float32).cuda(), S0.cuda()
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("B,T,H,dk", [(2, 150, 3, 64), (1, 64, 2, 128), (1, 1, 2, 128), (2, 200, 2, 128)])
+def test_gdn_chunk_vs_recurrence(cuda, dtype, B, T, H, dk):
+    import looped_hybrid_attention_b200 as L
+    q, k, v, g, beta, S = _gdn_inputs(B, T, H, dk, dk, dtype, seed=T + H)
+    S0 = S.clone()
+    out = torch.empty_like(v)
+    scale = 1.0 / np.sqrt(dk)
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale)
+    tol = TOL[dtype]
+    for b in range(B):
+        o_ref, S_ref = ops.gdn_recurrent(to64(q[b]), to64(k[b]), to64(v[b]), to64(g[b]), to64(beta[b]),
+                                         to64(S0[b]), scale)
+        assert rel_l2(to64(out[b]), o_ref) < tol
+        assert rel_l2(to64(S[b]), S_ref) < (1e-5 if dtype == "fp32" else 1e-4)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_gdn_step_and_chunk_continue(cuda, dtype):
+    """Chunked prefill of T tokens then single-token steps equals the recurrence over T + 3 tokens."""
+    import looped_hybrid_attention_b200 as L
+    B, T, H, dk = 3, 70, 4, 128
+    q, k, v, g, beta, S = _gdn_inputs(B, T + 3, H, dk, dk, dtype, seed=5)
+    S0 = S.clone()
+    out = torch.empty((B, T, H, dk), dtype=DT[dtype], device=cuda)
+    scale = 1.0 / np.sqrt(dk)
+    L.gdn_chunk_fwd(q[:, :T].contiguous(), k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(),
+                    beta[:, :T].contiguous(), S, out, scale)
+    o_steps = []
+    for t in range(T, T + 3):
+        ot = torch.empty((B, H, dk), dtype=DT[dtype], device=cuda)
+        L.gdn_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), g[:, t].contiguous(),
+                   beta[:, t].contiguous(), S, ot, scale)
+        o_steps.append(ot)
+    for b in range(B):
+        o_ref, S_ref = ops.gdn_recurrent(to64(q[b]), to64(k[b]), to64(v[b]), to64(g[b]), to64(beta[b]),
+                                         to64(S0[b]), scale)
+        got = np.concatenate([to64(out[b, :T])] + [to64(o[b])[None] for o in o_steps])
+        assert rel_l2(got, o_ref) < TOL[dtype]
+        assert rel_l2(to64(S[b]), S_ref) < (1e-5 if dtype == "fp32" else 1e-4)
+
+
+def test_gdn_special_cases(cuda):
+    import looped_hybrid_attention_b200 as L
+    B, T, H, dk = 1, 100, 2, 64
+    q, k, v, g, beta, S = _gdn_inputs(B, T, H, dk, dk, "fp32", seed=9)
+    S0 = S.clone()
+    out = torch.empty_like(v)
+    # decay 1 (g = 0) and beta = 0 leave the state unchanged; o = scale S0 q
+    L.gdn_chunk_fwd(q, k, v, torch.zeros_like(g), torch.zeros_like(beta), S, out, 0.5)
+    assert torch.allclose(S, S0, rtol=0, atol=1e-6)
+    ref = 0.5 * np.einsum("hij,thj->thi", to64(S0[0]), to64(q[0]))
+    assert rel_l2(to64(out[0]), ref) < 1e-5
+    # T = 0: nothing changes
+    L.gdn_chunk_fwd(q[:, :0], k[:, :0], v[:, :0], g[:, :0], beta[:, :0], S, out[:, :0], 0.5)
+    assert torch.equal(S, S0)
+
+
+def test_gdn_prep(cuda):
+    import looped_hybrid_attention_b200 as L
+    M, H, dk, dv = 50, 16, 128, 128
+    n_in = 2 * H * dk + H * dv + 2 * H
+    P = rnd((M, n_in), 20, "P", dtype="bf16")
+    ab, bb = rnd((H,), 21, "ab"), rnd((H,), 22, "bb")
+    q = torch.empty((M, H, dk), dtype=torch.bfloat16, device=cuda)
+    k, v = torch.empty_like(q), torch.empty((M, H, dv), dtype=torch.bfloat16, device=cuda)
+    g, beta = torch.empty((M, H), device=cuda), torch.empty((M, H), device=cuda)
+    L.gdn_prep(P, ab, bb, q, k, v, g, beta, H, dk, dv, 1e-6)
+    rq, rk, rv, ra, rb = ops.gdn_split_projection(to64(P), H, dk, dv)
+    assert rel_l2(to64(q), ops.l2norm(rq, 1e-6)) < TOL["bf16"]
+    assert rel_l2(to64(k), ops.l2norm(rk, 1e-6)) < TOL["bf16"]
+    assert np.array_equal(to64(v), rv)
+    gr, br = ops.gdn_gates(ra, rb, to64(ab), to64(bb))
+    assert rel_l2(to64(g), gr) < 1e-5 and rel_l2(to64(beta), br) < 1e-5
+
+
+@pytest.mark.slow
+def test_gdn_chunk_full_length_sampled_heads(cuda):
+    """The bench's shape (T = 8192, 16 heads x 128, bf16): heads 0 and 15 against the recurrence."""
+    import looped_hybrid_attention_b200 as L
+    B, T, H, dk = 1, 8192, 16, 128
+    q, k, v, g, beta, S = _gdn_inputs(B, T, H, dk, dk, "bf16", seed=77)
+    S0 = S.clone()
+    out = torch.empty_like(v)
+    scale = 1.0 / np.sqrt(dk)
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale)
+    for h in (0, 15):
+        sl = slice(h, h + 1)
+        o_ref, S_ref = ops.gdn_recurrent(to64(q[0, :, sl]), to64(k[0, :, sl]), to64(v[0, :, sl]), to64(g[0, :, sl]),
+                                         to64(beta[0, :, sl]), to64(S0[0, sl]), scale)
+        assert rel_l2(to64(out[0, :, sl]), o_ref) < TOL["bf16"]
+        assert rel_l2(to64(S[0, sl]), S_ref) < 1e-4
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _fa_case(B, T, Hq, Hkv, dh, dtype, seed):
+    n_in = 2 * Hq * dh + 2 * Hkv * dh
+    P = rnd((B * T, n_in), seed, "Pfa", dtype=dtype)
+    qn = rnd((dh,), seed, "qn", std=0.1, dtype=dtype) + 1
+    kn = rnd((dh,), seed, "kn", std=0.1, dtype=dtype) + 1
+    return P, qn, kn
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("B,T,Hq,Hkv,dh,rot,pos0", [(1, 70, 4, 1, 64, 16, 0), (2, 33, 16, 4, 256, 64, 5),
+                                                    (1, 130, 16, 4, 256, 64, 0)])
+def test_fa_prep_and_attention(cuda, dtype, B, T, Hq, Hkv, dh, rot, pos0):
+    import looped_hybrid_attention_b200 as L
+    eps, base = 1e-6, 10000.0
+    cap = pos0 + T + 7
+    P, qn, kn = _fa_case(B, T, Hq, Hkv, dh, dtype, seed=T)
+    qo = torch.empty((B * T, Hq, dh), dtype=DT[dtype], device=cuda)
+    Kc = torch.zeros((B, Hkv, cap, dh), dtype=DT[dtype], device=cuda)
+    Vc = torch.zeros_like(Kc)
+    if pos0:      # earlier tokens already in the slab
+        Kc[:, :, :pos0] = rnd((B, Hkv, pos0, dh), 99, "Kprev", dtype=dtype).to(DT[dtype])
+        Vc[:, :, :pos0] = rnd((B, Hkv, pos0, dh), 98, "Vprev", dtype=dtype).to(DT[dtype])
+    L.fa_prep(P, qn, kn, qo, Kc, Vc, cap, B, T, pos0, Hq, Hkv, dh, rot, base, eps)
+    tol = TOL[dtype]
+    Pn = to64(P).reshape(B, T, -1)
+    for b in range(B):
+        q, gate, k, v = ops.fa_split_projection(Pn[b], Hq, Hkv, dh)
+        rq, rk = ops.fa_qk(q, k, to64(qn), to64(kn), pos0 + np.arange(T), rot, base, eps)
+        assert rel_l2(to64(qo.view(B, T, Hq, dh)[b]), rq) < tol
+        assert rel_l2(to64(Kc[b, :, pos0:pos0 + T]).transpose(1, 0, 2), rk) < tol
+        assert np.array_equal(to64(Vc[b, :, pos0:pos0 + T]).transpose(1, 0, 2), v)
+    # attention with the gate, reading q from the compact buffer and the gate from P
+    out = torch.empty((B * T, Hq * dh), dtype=DT[dtype], device=cuda)
+    gate_view = P[:, Hq * dh:]
+    ws = torch.empty(max(1, L.gqa_workspace_bytes(B, T, pos0 + T, Hq, dh) // 4), device=cuda)
+    for workspace in (None, ws):
+        L.gqa_attn(qo, Hq * dh, Kc, Vc, cap, gate_view, P.stride(0), out, B, T, pos0 + T, pos0, Hq, Hkv, dh,
+                   True, workspace)
+        for b in range(B):
+            qb = to64(qo.view(B, T, Hq, dh)[b])
+            K = to64(Kc[b, :, :pos0 + T]).transpose(1, 0, 2)
+            V = to64(Vc[b, :, :pos0 + T]).transpose(1, 0, 2)
+            ref = ops.attention(qb, K, V, pos0 + np.arange(T))
+            _, gate, _, _ = ops.fa_split_projection(Pn[b], Hq, Hkv, dh)
+            ref = ref * ops.sigmoid(gate)
+            assert rel_l2(to64(out.view(B, T, Hq, dh)[b]), ref) < tol
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_decode_attention_split_k(cuda, dtype):
+    """One query per sequence over a long slab: split-K partials + combine (with workspace) equal brute force."""
+    import looped_hybrid_attention_b200 as L
+    B, Hq, Hkv, dh, L_ctx = 4, 16, 4, 256, 3000
+    cap = L_ctx + 10
+    q = rnd((B, Hq, dh), 30, "qd", dtype=dtype)
+    Kc = rnd((B, Hkv, cap, dh), 31, "Kd", dtype=dtype)
+    Vc = rnd((B, Hkv, cap, dh), 32, "Vd", dtype=dtype)
+    out = torch.empty((B, Hq * dh), dtype=DT[dtype], device=cuda)
+    ws = torch.empty(L.gqa_workspace_bytes(B, 1, L_ctx, Hq, dh) // 4 + 1, device=cuda)
+    L.gqa_attn(q, Hq * dh, Kc, Vc, cap, None, 0, out, B, 1, L_ctx, L_ctx - 1, Hq, Hkv, dh, True, ws)
+    for b in range(B):
+        ref = ops.attention(to64(q[b])[None], to64(Kc[b, :, :L_ctx]).transpose(1, 0, 2),
+                            to64(Vc[b, :, :L_ctx]).transpose(1, 0, 2), [L_ctx - 1])
+        assert rel_l2(to64(out[b]).reshape(1, Hq, dh), ref) < TOL[dtype]
+
+
+def test_attention_single_key_and_zero_query(cuda):
+    import looped_hybrid_attention_b200 as L
+    Hq, Hkv, dh, T = 4, 1, 64, 20
+    Kc = rnd((1, Hkv, T, dh), 40, "K1")
+    Vc = rnd((1, Hkv, T, dh), 41, "V1")
+    q = torch.zeros((T, Hq, dh), device=cuda)
+    out = torch.empty((T, Hq * dh), device=cuda)
+    L.gqa_attn(q, Hq * dh, Kc, Vc, T, None, 0, out, 1, T, T, 0, Hq, Hkv, dh, True)
+    mean = torch.cumsum(Vc[0, 0], 0) / torch.arange(1, T + 1, device=cuda)[:, None]
+    assert torch.allclose(out.view(T, Hq, dh), mean[:, None, :].expand(T, Hq, dh), atol=1e-5)
+    assert torch.allclose(out.view(T, Hq, dh)[0], Vc[0, 0, 0][None].expand(Hq, dh), atol=1e-6)
+
+
+@pytest.mark.slow
+def test_attention_full_length_sampled_rows(cuda):
+    """The bench's shape (T = 8192, 16q/4kv x 256, bf16): sampled query rows against brute force."""
+    import looped_hybrid_attention_b200 as L
+    T, Hq, Hkv, dh = 8192, 16, 4, 256
+    q = rnd((T, Hq, dh), 50, "qf", dtype="bf16")
+    Kc = rnd((1, Hkv, T, dh), 51, "Kf", dtype="bf16")
+    Vc = rnd((1, Hkv, T, dh), 52, "Vf", dtype="bf16")
+    out = torch.empty((T, Hq * dh), dtype=torch.bfloat16, device=cuda)
+    L.gqa_attn(q, Hq * dh, Kc, Vc, T, None, 0, out, 1, T, T, 0, Hq, Hkv, dh, True)
+    rows = np.array([0, 1, 63, 64, 127, 128, 4095, 5000, 8190, 8191])
+    ref = ops.attention(to64(q[rows]), to64(Kc[0]).transpose(1, 0, 2), to64(Vc[0]).transpose(1, 0, 2), rows)
+    assert rel_l2(to64(out[rows]).reshape(len(rows), Hq, dh), ref) < TOL["bf16"]
+
+
+# the projections of the 9B-shape prefill at T = 8192: (N, K, epilogue)
+FULL_GEMMS = [(6176, 4096, "store"), (2048 * 2, 2048, "store"), (10240, 4096, "store"), (4096, 4096, "store"),
+              (12288, 4096, "swiglu"), (4096, 12288, "add")]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("N,K,epi", FULL_GEMMS)
+def test_linear_full_size_sampled_rows(cuda, N, K, epi):
+    """bf16 projections at M = 8192 (the prefill bench's token count): sampled rows vs fp64."""
+    import looped_hybrid_attention_b200 as L
+    M = 8192
+    X = torch.randn((M, K), device=cuda, generator=torch.Generator(device=cuda).manual_seed(1)).to(torch.bfloat16)
+    W = (0.02 * torch.randn((N, K), device=cuda, generator=torch.Generator(device=cuda).manual_seed(2))).to(torch.bfloat16)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=cuda)
+    rows = np.array([0, 1, 127, 128, 129, 4000, 8063, 8064, 8190, 8191])
+    xr = to64(X[rows])
+    if epi == "swiglu":
+        W2 = (0.02 * torch.randn((N, K), device=cuda, generator=torch.Generator(device=cuda).manual_seed(3))).to(torch.bfloat16)
+        L.linear(X, W, Y, L.EPI_SWIGLU, W2=W2)
+        ref = ops.silu(ops.linear(xr, to64(W))) * ops.linear(xr, to64(W2))
+    elif epi == "add":
+        R = torch.randn((M, N), device=cuda, generator=torch.Generator(device=cuda).manual_seed(4)).to(torch.bfloat16)
+        L.linear(X, W, Y, L.EPI_ADD, R=R)
+        ref = ops.linear(xr, to64(W)) + to64(R[rows])
+    else:
+        L.linear(X, W, Y, L.EPI_STORE)
+        ref = ops.linear(xr, to64(W))
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert rel_l2(to64(Y[rows]), ref) < TOL["bf16"]
+    # every row is written (no tile skipped): compare row norms against a cheap fp32 reference
+    if epi == "store":
+        ref_all = (X.float() @ W.float().t())
+        assert rel_l2(to64(Y), to64(ref_all)) < TOL["bf16"]
+
+
+def test_lm_head_shape_fp32_out(cuda):
+    """M = 1..64 rows (prefill last position / decode batch) against the 248,320-row LM head, fp32 logits."""
+    import looped_hybrid_attention_b200 as L
+    V, d = 248320, 4096
+    W = (0.02 * torch.randn((V, d), device=cuda, generator=torch.Generator(device=cuda).manual_seed(5))).to(torch.bfloat16)
+    for M in (1, 64):
+        X = torch.randn((M, d), device=cuda, generator=torch.Generator(device=cuda).manual_seed(6)).to(torch.bfloat16)
+        Y = torch.empty((M, V), device=cuda)
+        L.linear(X, W, Y, L.EPI_F32)
+        cols = np.r_[0:64, 124000:124100, V - 70:V]
+        ref = ops.linear(to64(X), to64(W[cols]))
+        assert rel_l2(to64(Y[:, cols]), ref) < 1e-4
