@@ -1,0 +1,321 @@
+"""Benchmark: prefill of the 56-execution looped hybrid stack (9B shape, bf16) on B200.
+
+Workload (default): the full 9B-shape stack with random-init bf16 weights -- vocab
+248,320 embedding + LM head, 32 stored layers run as 56 executions (4 + 24x2 + 4),
+hidden 4096, FFN 12288, 3:1 GDN/GQA groups, two-stream mHC with FP32 routing --
+prefill of batch 1 x 8192 uniform random token ids.  One step = one prefill (all
+56 executions, final norm, LM head on the last position) from an empty cache.
+
+`python bench.py [--gpus N --steps K --warmup W]` prints one JSON line.  With
+--gpus N > 1 it runs under torchrun as N independent replicas (the forward pass
+has no exchange step), one process per GPU; time is the max over ranks.
+`--impl reference` times the CPU oracle instead, on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SEQ, BATCH = 8192, 1
+WORKLOAD = "9B-shape looped hybrid stack, 56 executions, prefill B=1 T=8192, bf16, random-init weights"
+
+
+def load_peaks():
+    """Measured B200 peaks of this machine (driver-written), else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device):
+        import torch
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.index = str(device.index or 0)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(T=64, seed=0):
+    """The CPU oracle on a bounded sample of the workload: one full-width group (3 GDN + 1 GQA
+    layers inside the two-stream mHC) on T tokens.  Returns (seconds, tokens, executions)."""
+    import numpy as np
+    import torch
+
+    import synth
+    from oracle import model as omodel
+    s = synth.GROUP
+    W = omodel.Weights(synth.make_weights(s, seed=seed))
+    for name, _, _ in synth.weight_names(s):      # widen the weights before timing (not oracle work)
+        W[name]
+    h = synth.normal((1, T, s.d), 1.0, seed, "hidden").to(torch.bfloat16)
+    t0 = time.perf_counter()
+    omodel.forward_hidden(s, W, h)
+    dt = time.perf_counter() - t0
+    return dt, T, 4
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+        return int(n)
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline_entry(T=64):
+    dt, tokens, execs = oracle_sample(T)
+    # per-token time of the full stack = (time per execution per token) x 56 executions
+    per_token = dt / tokens / execs * 56
+    return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"oracle forward of one full-width group (3 GDN + 1 GQA + mHC, d 4096) on {tokens} tokens "
+                      f"({dt:.2f} s), scaled to 56 executions per token; LM head excluded"}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(args.ref_tokens)
+    times = []
+    for _ in range(args.steps):
+        dt, tokens, execs = oracle_sample(args.ref_tokens)
+        times.append(dt / tokens / execs * 56)
+    value = 1.0 / (sum(times) / len(times))
+    line = {"impl": "reference", "metric": "prefill tokens/s (56-execution looped hybrid stack)", "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * sum(times) / len(times) * SEQ, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": SEQ, "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": f"each step: oracle forward of one full-width group on {args.ref_tokens} "
+                                       "tokens, scaled to 56 executions per token"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import looped_hybrid_attention_b200 as L
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    s = synth.FULL
+    w = synth.make_weights(s, seed=args.seed + rank, device=dev)
+    m = L.Model(s, w)
+    c = m.cache(BATCH, SEQ)
+    ids = synth.uniform_ids((BATCH, SEQ), s.vocab, args.seed + rank, device=dev)
+    logits = torch.empty((BATCH, s.vocab), device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        c.reset()
+        m.prefill(c, ids, logits, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert torch.isfinite(logits).all(), "non-finite logits"
+
+    # ---------------- device-resident timed region (with per-kernel events)
+    m.profile(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    kernels = m.profile_read()
+    m.profile(False)
+    ms = max_over_ranks(ms, world)
+    tokens = BATCH * SEQ * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # ---------------- end to end through the public API with host buffers
+    ids_host = ids.cpu().pin_memory()
+    logits_host = torch.empty((BATCH, s.vocab), pin_memory=True)
+    ids_dev = torch.empty_like(ids)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        ids_dev.copy_(ids_host, non_blocking=True)
+        c.reset()
+        m.prefill(c, ids_dev, logits, stream)
+        logits_host.copy_(logits, non_blocking=True)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    peaks = load_peaks()
+    top = max(kernels.items(), key=lambda kv: kv[1]["ms"])
+    name, k = top
+    per_launch_ms = k["ms"] / k["launches"]
+    if k["flops"] > 0 and name in ("gemm", "attention", "gdn_chunk"):
+        achieved = k["flops"] / (k["ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained (" + peaks["source"] + ")"}
+    else:
+        achieved = k["bytes"] / (k["ms"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + peaks["source"] + ")"}
+    roof.update({"kernel": name, "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
+                 "launches": k["launches"], "ms_per_launch": round(per_launch_ms, 4),
+                 "algorithmic_per_launch": (k["flops"] if roof["bound"] == "tensor" else k["bytes"]) / k["launches"],
+                 "traffic": None})
+    per_kernel = {}
+    total_ms = sum(v["ms"] for v in kernels.values())
+    for kname, v in sorted(kernels.items(), key=lambda kv: -kv[1]["ms"]):
+        e = {"launches": v["launches"] // args.steps, "ms_per_step": round(v["ms"] / args.steps, 3),
+             "share": round(v["ms"] / total_ms, 4)}
+        if v["flops"]:
+            e["tflops"] = round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)
+        if v["bytes"]:
+            e["gbs"] = round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)
+        per_kernel[kname] = e
+    launches = sum(v["launches"] for v in kernels.values())
+
+    if rank != 0:
+        return
+    line = {"metric": "prefill tokens/s (56-execution looped hybrid stack)", "value": round(value, 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, uniform token ids)",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": SEQ,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (16.3 GB of weights streamed per step)"},
+            "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": ids.numel() * 4, "d2h_bytes_per_step": logits.numel() * 4},
+            "gpu_launches": launches, "roofline": roof, "kernels": per_kernel,
+            "clocks": clk.summary()}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_entry(args.ref_tokens)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-tokens", type=int, default=64, help="tokens per oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = 1, int(os.environ.get("RANK", "0")), 0
+    if args.impl == "ours":
+        world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -254,6 +254,25 @@ loop_status loop_embed(const int32_t* ids, const void* embed, void* out, int M, 
 /* next [B] int32 = argmax over logits [B, V] fp32, lowest index on ties. */
 loop_status loop_argmax(const float* logits, int32_t* next, int B, int V, void* stream);
 
+/* ---------------------------------------------------------------- per-kernel timing
+ * While enabled, the model brackets every kernel launch of loop_prefill /
+ * loop_forward_hidden / loop_decode_step with CUDA events on the launch stream and
+ * records the launch's algorithmic work (flops = 2 x multiply-adds of the definition;
+ * bytes = the tensors the kernel must read and write once).  loop_profile_read
+ * synchronises on the recorded events and returns one entry per kernel class
+ * ("gemm", "lm_head", "gdn_chunk", "gdn_step", "attention", "mhc", ...), summed over
+ * everything recorded since loop_profile_enable(m, 1).  Events add a few microseconds
+ * of host time per launch. */
+typedef struct loop_profile_entry {
+  char name[24];
+  int launches;       /* kernel launches of this class */
+  double ms;          /* summed event time */
+  double flops;       /* summed algorithmic flops */
+  double bytes;       /* summed algorithmic HBM bytes */
+} loop_profile_entry;
+loop_status loop_profile_enable(loop_model* m, int on);
+loop_status loop_profile_read(loop_model* m, loop_profile_entry* out /* host [cap] */, int cap, int* n /* host */);
+
 #ifdef __cplusplus
 }
 #endif

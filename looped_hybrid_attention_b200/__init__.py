@@ -48,6 +48,11 @@ class loop_layer_weights(ctypes.Structure):
         "w_gate", "w_up", "w_down", "mhc_w_r", "mhc_b_r")]
 
 
+class loop_profile_entry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("launches", ctypes.c_int), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 class loop_weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
                 ("layers", ctypes.POINTER(loop_layer_weights)), ("n_layers", ctypes.c_int)]
@@ -83,6 +88,8 @@ _SIGS = {
     "loop_rmsnorm": ([_P] * 5 + [_I, _I, _F, _I, _P], _I),
     "loop_embed": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
     "loop_argmax": ([_P, _P, _I, _I, _P], _I),
+    "loop_profile_enable": ([_P, _I], _I),
+    "loop_profile_read": ([_P, _P, _I, ctypes.POINTER(ctypes.c_int)], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -196,6 +203,18 @@ class Model:
             self.handle = None
 
     __del__ = close
+
+    def profile(self, on=True):
+        """Start (clearing) or stop per-kernel event timing inside the model's launches."""
+        check(_lib.loop_profile_enable(self.handle, int(on)), "loop_profile_enable")
+
+    def profile_read(self):
+        """{kernel class: {launches, ms, flops, bytes}} summed since profile(True)."""
+        buf = (loop_profile_entry * 32)()
+        n = ctypes.c_int(0)
+        check(_lib.loop_profile_read(self.handle, buf, 32, ctypes.byref(n)), "loop_profile_read")
+        return {buf[i].name.decode(): {"launches": buf[i].launches, "ms": buf[i].ms, "flops": buf[i].flops,
+                                       "bytes": buf[i].bytes} for i in range(min(n.value, 32))}
 
     def cache(self, batch, max_tokens):
         return Cache(self, batch, max_tokens)

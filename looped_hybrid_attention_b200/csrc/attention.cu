@@ -256,6 +256,10 @@ size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
   return (size_t)B * Tq * Hq * s * (dh + 2) * sizeof(float);
 }
 
+int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace) {
+  return has_workspace && attn_splits(B, Tq, Tkv, Hkv) > 1 ? 2 : 1;
+}
+
 bool gqa_supported(int dh, int Hq, int Hkv) {
   return (dh == 64 || dh == 128 || dh == 256) && Hkv > 0 && Hq % Hkv == 0 && Hq / Hkv <= 32;
 }

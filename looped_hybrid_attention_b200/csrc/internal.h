@@ -47,6 +47,7 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                      cudaStream_t s);
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
 bool gqa_supported(int dh, int Hq, int Hkv);
+int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace);
 
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
                 const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,

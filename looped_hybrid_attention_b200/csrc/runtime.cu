@@ -6,6 +6,7 @@
 // execution, pre-norm mixer + SwiGLU FFN; inside the loop block the two-stream mHC
 // kernel runs once per layer boundary (open -> mix+route ... -> merge, §六).
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -36,6 +37,53 @@ cudaError_t DevBuf::ensure(size_t want) {
   cudaError_t e = cudaMalloc(&p, want);
   if (e == cudaSuccess) bytes = want;
   return e;
+}
+
+const char* const kProfNames[P_NCAT] = {"gemm", "lm_head", "rmsnorm", "embed", "gdn_prep", "gdn_chunk", "gdn_step",
+                                        "fa_prep", "attention", "mhc", "argmax", "copy"};
+
+Profiler::~Profiler() {
+  clear();
+  for (auto e : pool) cudaEventDestroy(e);
+}
+cudaEvent_t Profiler::get() {
+  if (pool.empty()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+  cudaEvent_t e = pool.back();
+  pool.pop_back();
+  return e;
+}
+void Profiler::clear() {
+  for (auto& r : recs) {
+    pool.push_back(r.a);
+    pool.push_back(r.b);
+  }
+  recs.clear();
+}
+
+// Run `launch` (returns cudaError_t); with profiling on, bracket it with events and
+// record its algorithmic work.
+template <typename F>
+static cudaError_t prof(loop_model* m, cudaStream_t s, int cat, int launches, double flops, double bytes, F&& launch) {
+  if (!m->prof.on) return launch();
+  ProfRec r{cat, launches, m->prof.get(), m->prof.get(), flops, bytes};
+  if (!r.a || !r.b) return cudaErrorMemoryAllocation;
+  cudaEventRecord(r.a, s);
+  cudaError_t e = launch();
+  cudaEventRecord(r.b, s);
+  m->prof.recs.push_back(r);
+  return e;
+}
+
+// Algorithmic work of one projection launch (bf16 or fp32 storage).
+static void gemm_work(long M, long N, long K, int epi, size_t es, double& flops, double& bytes) {
+  const long n_mat = epi == EPI_SWIGLU ? 2 : 1;
+  flops = 2.0 * M * N * K * n_mat;
+  bytes = (double)es * (M * K + n_mat * N * K) + (epi == EPI_F32 ? 4.0 : (double)es) * M * N +
+          (epi == EPI_ADD ? (double)es * M * N : 0.0);
 }
 
 std::vector<ExecRow> build_schedule(const loop_config& c) {
@@ -104,51 +152,88 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
   const loop_layer_weights& w = m->layers[r.layer];
   const long M = (long)B * T;
   const int d = cf.d, dt = cf.dtype;
-  CK(rmsnorm(x, nullptr, nullptr, w.attn_norm, m->xn.p, (int)M, d, cf.eps, dt, s), "rmsnorm (mixer)");
+  const double es = (double)m->esize;
+  double fl, by;
+  CK(prof(m, s, P_RMSNORM, 1, 0, es * (2.0 * M * d + d),
+          [&] { return rmsnorm(x, nullptr, nullptr, w.attn_norm, m->xn.p, (int)M, d, cf.eps, dt, s); }),
+     "rmsnorm (mixer)");
   if (r.kind == 0) {
     const int H = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
-    CK(linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d, EPI_STORE, dt, s),
+    gemm_work(M, m->in_gdn, d, EPI_STORE, m->esize, fl, by);
+    CK(prof(m, s, P_GEMM, 1, fl, by,
+            [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d,
+                                EPI_STORE, dt, s); }),
        "GDN input projection");
-    CK(lk::gdn_prep(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p,
-                (float*)m->gb.p, (int)M, H, dk, dv, cf.eps, dt, s),
+    CK(prof(m, s, P_GDN_PREP, 1, 0, (double)M * (es * (m->in_gdn + 2.0 * H * dk + H * dv) + 8.0 * H),
+            [&] { return lk::gdn_prep(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p,
+                                      (float*)m->gg.p, (float*)m->gb.p, (int)M, H, dk, dv, cf.eps, dt, s); }),
        "GDN prep");
     float* S = (float*)c->state.p + (size_t)r.slot * c->state_elems;
     const float scale = 1.f / std::sqrt((float)dk);
+    // bytes: q, k, v in, o out, gates, and the fp32 state read + written once
+    const double st_bytes = 8.0 * B * H * dk * dv;
+    const double io_bytes = (double)M * H * (es * (2.0 * dk + 2.0 * dv) + 8.0);
     if (T == 1)
-      CK(lk::gdn_step(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, H, dk, dv, scale, dt, s),
+      CK(prof(m, s, P_GDN_STEP, 1, 6.0 * B * H * dk * dv, io_bytes + st_bytes,
+              [&] { return lk::gdn_step(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, H,
+                                        dk, dv, scale, dt, s); }),
          "GDN step");
-    else
-      CK(gdn_chunk(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, T, H, dk, dv, scale,
-                   dt, s),
+    else {
+      // flops of the chunked form per 64-token chunk and head (A and P, substitution, U, O, state)
+      const double C = 64.0, chunks = (double)B * H * ((T + 63) / 64);
+      const double per_chunk = 2.0 * C * C * dk + C * C * (dk + dv) + 2.0 * C * dk * dv * 3 + C * C * dv;
+      CK(prof(m, s, P_GDN_CHUNK, 1, chunks * per_chunk, io_bytes + st_bytes,
+              [&] { return gdn_chunk(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, T, H,
+                                     dk, dv, scale, dt, s); }),
          "GDN chunked scan");
-    CK(linear(m->o.p, H * dv, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, H * dv, EPI_STORE, dt, s),
+    }
+    gemm_work(M, d, H * dv, EPI_STORE, m->esize, fl, by);
+    CK(prof(m, s, P_GEMM, 1, fl, by,
+            [&] { return linear(m->o.p, H * dv, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, H * dv, EPI_STORE,
+                                dt, s); }),
        "GDN output projection");
   } else {
     const int Hq = cf.fa_q_heads, Hkv = cf.fa_kv_heads, dh = cf.fa_head_dim;
-    CK(linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d, EPI_STORE, dt, s),
+    gemm_work(M, m->in_fa, d, EPI_STORE, m->esize, fl, by);
+    CK(prof(m, s, P_GEMM, 1, fl, by,
+            [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d,
+                                EPI_STORE, dt, s); }),
        "FA input projection");
     char* kbase = (char*)c->kv.p + (size_t)r.slot * 2 * c->kv_slab_elems * m->esize;
     char* vbase = kbase + c->kv_slab_elems * m->esize;
-    CK(lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, m->gq.p, kbase, vbase, c->max_tokens, B, T, pos0, Hq, Hkv, dh,
-               cf.rotary_dims, cf.rope_base, cf.eps, dt, s),
+    CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * (Hq + 2 * Hkv) * dh),
+            [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, m->gq.p, kbase, vbase, c->max_tokens, B, T,
+                                     pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt, s); }),
        "QK-norm / rotary / KV write");
     const char* gate = (const char*)m->proj.p + (size_t)Hq * dh * m->esize;
-    CK(lk::gqa_attn(m->gq.p, Hq * dh, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B, T, pos0 + T, pos0, Hq, Hkv,
-                dh, 1, m->attn_ws.p, dt, s),
+    // causal (query, key) pairs: sum over new tokens of (pos0 + t + 1)
+    const double pairs = (double)B * ((double)T * pos0 + (double)T * (T + 1) / 2.0);
+    const double attn_bytes = es * ((double)M * Hq * dh * 3.0 + (double)B * Hkv * (pos0 + T) * dh * 2.0);
+    CK(prof(m, s, P_ATTN, gqa_launches(B, T, pos0 + T, Hkv, m->attn_ws.p != nullptr), 4.0 * Hq * dh * pairs, attn_bytes,
+            [&] { return lk::gqa_attn(m->gq.p, Hq * dh, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B, T,
+                                      pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s); }),
        "GQA attention");
-    CK(linear(m->o.p, Hq * dh, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, Hq * dh, EPI_STORE, dt, s),
+    gemm_work(M, d, Hq * dh, EPI_STORE, m->esize, fl, by);
+    CK(prof(m, s, P_GEMM, 1, fl, by,
+            [&] { return linear(m->o.p, Hq * dh, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, Hq * dh,
+                                EPI_STORE, dt, s); }),
        "FA output projection");
   }
   // u = x + mix; FFN on RMSNorm(u)
-  CK(rmsnorm(x, m->mix.p, m->u.p, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s), "rmsnorm (FFN)");
-  CK(linear(m->un.p, d, w.w_gate, w.w_up, nullptr, 0, m->act.p, cf.ffn, (int)M, cf.ffn, d, EPI_SWIGLU, dt, s),
+  CK(prof(m, s, P_RMSNORM, 1, 0, es * (4.0 * M * d + d),
+          [&] { return rmsnorm(x, m->mix.p, m->u.p, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s); }),
+     "rmsnorm (FFN)");
+  gemm_work(M, cf.ffn, d, EPI_SWIGLU, m->esize, fl, by);
+  CK(prof(m, s, P_GEMM, 1, fl, by,
+          [&] { return linear(m->un.p, d, w.w_gate, w.w_up, nullptr, 0, m->act.p, cf.ffn, (int)M, cf.ffn, d, EPI_SWIGLU,
+                              dt, s); }),
      "FFN gate/up (SwiGLU)");
-  if (r.in_loop)
-    CK(linear(m->act.p, cf.ffn, w.w_down, nullptr, m->mix.p, d, m->F.p, d, (int)M, d, cf.ffn, EPI_ADD, dt, s),
-       "FFN down (+ mixer output)");
-  else
-    CK(linear(m->act.p, cf.ffn, w.w_down, nullptr, m->u.p, d, h_out, d, (int)M, d, cf.ffn, EPI_ADD, dt, s),
-       "FFN down (+ residual)");
+  gemm_work(M, d, cf.ffn, EPI_ADD, m->esize, fl, by);
+  const void* res = r.in_loop ? m->mix.p : m->u.p;
+  void* dst = r.in_loop ? m->F.p : h_out;
+  CK(prof(m, s, P_GEMM, 1, fl, by,
+          [&] { return linear(m->act.p, cf.ffn, w.w_down, nullptr, res, d, dst, d, (int)M, d, cf.ffn, EPI_ADD, dt, s); }),
+     "FFN down (+ residual)");
   return LOOP_OK;
 }
 
@@ -166,20 +251,25 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
       continue;
     }
     const loop_layer_weights& w = m->layers[r.layer];
+    const double es = (double)m->esize, tok = (double)M;
     if (r.exec == m->first_loop)
-      CK(mhc(MHC_OPEN, m->h.p, nullptr, nullptr, w.mhc_w_r, w.mhc_b_r, m->X.p, m->x_in.p, nullptr, (float*)m->coeffs.p,
-             (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s),
+      CK(prof(m, s, P_MHC, 1, 0, tok * (es * 4.0 * cf.d + 32.0),
+              [&] { return mhc(MHC_OPEN, m->h.p, nullptr, nullptr, w.mhc_w_r, w.mhc_b_r, m->X.p, m->x_in.p, nullptr,
+                               (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
          "mHC open");
     loop_status st = run_layer(m, c, r, m->x_in.p, nullptr, B, T, pos0, s);
     if (st != LOOP_OK) return st;
     if (r.exec == m->last_loop) {
-      CK(mhc(MHC_MERGE, m->X.p, m->F.p, (float*)m->coeffs.p, nullptr, nullptr, nullptr, nullptr, m->h.p, nullptr,
-             (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s),
+      CK(prof(m, s, P_MHC, 1, 0, tok * (es * 4.0 * cf.d + 32.0),
+              [&] { return mhc(MHC_MERGE, m->X.p, m->F.p, (float*)m->coeffs.p, nullptr, nullptr, nullptr, nullptr,
+                               m->h.p, nullptr, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
          "mHC merge");
     } else {
       const loop_layer_weights& wn = m->layers[m->sched[i + 1].layer];
-      CK(mhc(MHC_MIX, m->X.p, m->F.p, (float*)m->coeffs.p, wn.mhc_w_r, wn.mhc_b_r, m->X.p, m->x_in.p, nullptr,
-             (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s),
+      // read X (2d) + F (d), write X' (2d) + x_in (d), coefficients in/out
+      CK(prof(m, s, P_MHC, 1, 0, tok * (es * 6.0 * cf.d + 64.0),
+              [&] { return mhc(MHC_MIX, m->X.p, m->F.p, (float*)m->coeffs.p, wn.mhc_w_r, wn.mhc_b_r, m->X.p, m->x_in.p,
+                               nullptr, (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
          "mHC mix + route");
     }
   }
@@ -192,8 +282,11 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
   const long M = (long)B * T;
   loop_status st = ensure_workspace(m, M, B, T, c->max_tokens);
   if (st != LOOP_OK) return st;
+  const double es = (double)m->esize;
   if (ids)
-    CK(embed(ids, m->embed, m->h.p, (int)M, cf.d, cf.vocab, cf.dtype, s), "embedding");
+    CK(prof(m, s, P_EMBED, 1, 0, (double)M * (2.0 * es * cf.d + 4.0),
+            [&] { return embed(ids, m->embed, m->h.p, (int)M, cf.d, cf.vocab, cf.dtype, s); }),
+       "embedding");
   else
     CK(cudaMemcpyAsync(m->h.p, h_in, M * cf.d * m->esize, cudaMemcpyDeviceToDevice, s), "hidden-state input copy");
   st = run_stack(m, c, B, T, s);
@@ -203,10 +296,15 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
   if (logits_last) {
     // final norm of each sequence's last position, then the LM head
     const char* last = (const char*)m->h.p + (size_t)(T - 1) * cf.d * m->esize;
-    CK(rmsnorm(last, nullptr, nullptr, m->final_norm, m->last.p, B, cf.d, cf.eps, cf.dtype, s, (long)T * cf.d),
+    CK(prof(m, s, P_RMSNORM, 1, 0, es * (2.0 * B * cf.d + cf.d),
+            [&] { return rmsnorm(last, nullptr, nullptr, m->final_norm, m->last.p, B, cf.d, cf.eps, cf.dtype, s,
+                                 (long)T * cf.d); }),
        "final norm");
-    CK(linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, logits_last, cf.vocab, B, cf.vocab, cf.d, EPI_F32,
-              cf.dtype, s),
+    double fl, by;
+    gemm_work(B, cf.vocab, cf.d, EPI_F32, m->esize, fl, by);
+    CK(prof(m, s, P_LMHEAD, 1, fl, by,
+            [&] { return linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, logits_last, cf.vocab, B, cf.vocab,
+                                cf.d, EPI_F32, cf.dtype, s); }),
        "LM head");
   }
   return LOOP_OK;
@@ -225,13 +323,56 @@ loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* 
     CK(tmp.ensure((size_t)B * cf.vocab * sizeof(float)), "logits buffer");
     lg = (float*)tmp.p;
   }
-  CK(embed(tok, m->embed, m->h.p, B, cf.d, cf.vocab, cf.dtype, s), "embedding");
+  const double es = (double)m->esize;
+  CK(prof(m, s, P_EMBED, 1, 0, (double)B * (2.0 * es * cf.d + 4.0),
+          [&] { return embed(tok, m->embed, m->h.p, B, cf.d, cf.vocab, cf.dtype, s); }),
+     "embedding");
   st = run_stack(m, c, B, 1, s);
   if (st != LOOP_OK) return st;
   c->len += 1;
-  CK(rmsnorm(m->h.p, nullptr, nullptr, m->final_norm, m->last.p, B, cf.d, cf.eps, cf.dtype, s), "final norm");
-  CK(linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, lg, cf.vocab, B, cf.vocab, cf.d, EPI_F32, cf.dtype, s),
+  CK(prof(m, s, P_RMSNORM, 1, 0, es * (2.0 * B * cf.d + cf.d),
+          [&] { return rmsnorm(m->h.p, nullptr, nullptr, m->final_norm, m->last.p, B, cf.d, cf.eps, cf.dtype, s); }),
+     "final norm");
+  double fl, by;
+  gemm_work(B, cf.vocab, cf.d, EPI_F32, m->esize, fl, by);
+  CK(prof(m, s, P_LMHEAD, 1, fl, by,
+          [&] { return linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, lg, cf.vocab, B, cf.vocab, cf.d, EPI_F32,
+                              cf.dtype, s); }),
      "LM head");
-  CK(argmax(lg, next, B, cf.vocab, s), "argmax");
+  CK(prof(m, s, P_ARGMAX, 1, 0, 4.0 * B * cf.vocab + 4.0 * B, [&] { return argmax(lg, next, B, cf.vocab, s); }),
+     "argmax");
+  return LOOP_OK;
+}
+
+// ------------------------------------------------------------------ profiling ABI
+extern "C" loop_status loop_profile_enable(loop_model* m, int on) {
+  if (!m) return fail(LOOP_ERR_INVALID_ARG, "model is NULL");
+  m->prof.clear();
+  m->prof.on = on != 0;
+  return LOOP_OK;
+}
+
+extern "C" loop_status loop_profile_read(loop_model* m, loop_profile_entry* out, int cap, int* n) {
+  if (!m || !n) return fail(LOOP_ERR_INVALID_ARG, "NULL argument");
+  loop_profile_entry acc[P_NCAT];
+  memset(acc, 0, sizeof(acc));
+  for (int c = 0; c < P_NCAT; ++c) snprintf(acc[c].name, sizeof(acc[c].name), "%s", kProfNames[c]);
+  for (auto& r : m->prof.recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event");
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    acc[r.cat].launches += r.launches;
+    acc[r.cat].ms += ms;
+    acc[r.cat].flops += r.flops;
+    acc[r.cat].bytes += r.bytes;
+  }
+  int k = 0;
+  for (int c = 0; c < P_NCAT; ++c)
+    if (acc[c].launches) {
+      if (out && k < cap) out[k] = acc[c];
+      ++k;
+    }
+  *n = k;
   return LOOP_OK;
 }

@@ -22,6 +22,24 @@ struct DevBuf {
   cudaError_t ensure(size_t want);   // grow-only
 };
 
+// Per-launch event pairs with the launch's algorithmic work (enabled by loop_profile_enable).
+struct ProfRec {
+  int cat, launches;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;   // events ready for reuse
+  ~Profiler();
+  cudaEvent_t get();
+  void clear();
+};
+enum ProfCat { P_GEMM, P_LMHEAD, P_RMSNORM, P_EMBED, P_GDN_PREP, P_GDN_CHUNK, P_GDN_STEP, P_FA_PREP, P_ATTN, P_MHC,
+               P_ARGMAX, P_COPY, P_NCAT };
+extern const char* const kProfNames[P_NCAT];
+
 struct loop_model {
   loop_config cfg;
   std::vector<loop_layer_weights> layers;
@@ -36,6 +54,7 @@ struct loop_model {
   long ws_tokens = 0;
   DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, last;
   int in_gdn = 0, in_fa = 0;
+  Profiler prof;
 };
 
 struct loop_cache {

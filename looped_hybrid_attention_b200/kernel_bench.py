@@ -1,0 +1,98 @@
+"""Time one kernel of the library at a chosen shape (CUDA events), e.g. for ncu captures.
+
+  python -m looped_hybrid_attention_b200.kernel_bench gemm --M 8192 --N 12288 --K 4096 --epi swiglu
+  python -m looped_hybrid_attention_b200.kernel_bench gdn --T 8192 --H 16
+  python -m looped_hybrid_attention_b200.kernel_bench attn --T 8192
+  python -m looped_hybrid_attention_b200.kernel_bench mhc --T 8192
+
+Inputs are random bf16 tensors created on the device (larger than L2 at the default
+sizes); the printed rate uses the same algorithmic flop/byte counts as bench.py.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import looped_hybrid_attention_b200 as L
+
+
+def timed(fn, warmup, iters):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("op", choices=["gemm", "gdn", "attn", "mhc"])
+    ap.add_argument("--M", type=int, default=8192)
+    ap.add_argument("--N", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--epi", choices=["store", "add", "swiglu", "f32"], default="swiglu")
+    ap.add_argument("--T", type=int, default=8192)
+    ap.add_argument("--H", type=int, default=16)
+    ap.add_argument("--B", type=int, default=1)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--iters", type=int, default=10)
+    a = ap.parse_args()
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    bf = torch.bfloat16
+    r = lambda *s, std=1.0: (std * torch.randn(*s, device=dev, generator=g)).to(bf)
+    res = {"op": a.op}
+    if a.op == "gemm":
+        X, W = r(a.M, a.K), r(a.N, a.K, std=0.02)
+        W2 = r(a.N, a.K, std=0.02) if a.epi == "swiglu" else None
+        R = r(a.M, a.N) if a.epi == "add" else None
+        Y = torch.empty((a.M, a.N), device=dev, dtype=torch.float32 if a.epi == "f32" else bf)
+        epi = {"store": L.EPI_STORE, "add": L.EPI_ADD, "swiglu": L.EPI_SWIGLU, "f32": L.EPI_F32}[a.epi]
+        ms = timed(lambda: L.linear(X, W, Y, epi, W2=W2, R=R), a.warmup, a.iters)
+        flops = 2.0 * a.M * a.N * a.K * (2 if a.epi == "swiglu" else 1)
+        res.update(shape=[a.M, a.N, a.K], epi=a.epi, ms=ms, tflops=flops / ms / 1e9)
+    elif a.op == "gdn":
+        B, T, H, dk = a.B, a.T, a.H, 128
+        q = torch.nn.functional.normalize(torch.randn(B, T, H, dk, device=dev, generator=g), dim=-1).to(bf)
+        k = torch.nn.functional.normalize(torch.randn(B, T, H, dk, device=dev, generator=g), dim=-1).to(bf)
+        v = r(B, T, H, dk)
+        gg = -torch.nn.functional.softplus(torch.randn(B, T, H, device=dev, generator=g))
+        beta = torch.sigmoid(torch.randn(B, T, H, device=dev, generator=g))
+        S = torch.zeros(B, H, dk, dk, device=dev)
+        out = torch.empty_like(v)
+        ms = timed(lambda: L.gdn_chunk_fwd(q, k, v, gg, beta, S, out, dk ** -0.5), a.warmup, a.iters)
+        byts = B * T * H * (4 * dk * 2 + 8) + 8 * B * H * dk * dk
+        res.update(shape=[B, T, H, dk], ms=ms, gbs=byts / ms / 1e6)
+    elif a.op == "attn":
+        B, T, Hq, Hkv, dh = a.B, a.T, 16, 4, 256
+        q, gate = r(B * T, Hq, dh), r(B * T, Hq * dh)
+        K, V = r(B, Hkv, T, dh), r(B, Hkv, T, dh)
+        out = torch.empty((B * T, Hq * dh), device=dev, dtype=bf)
+        ms = timed(lambda: L.gqa_attn(q, Hq * dh, K, V, T, gate, Hq * dh, out, B, T, T, 0, Hq, Hkv, dh, True),
+                   a.warmup, a.iters)
+        flops = 4.0 * Hq * dh * B * T * (T + 1) / 2
+        res.update(shape=[B, T, Hq, Hkv, dh], ms=ms, tflops=flops / ms / 1e9)
+    else:
+        N, d = a.B * a.T, 4096
+        X, F = r(N, 2, d), r(N, d)
+        w_r = 0.02 * torch.randn(2 * d, 8, device=dev, generator=g)
+        b_r = torch.zeros(8, device=dev)
+        c_in = torch.tensor([0.5, 0.5, 1, 1, 0.6, 0.4, 0.4, 0.6], device=dev).repeat(N, 1)
+        c_out = torch.empty_like(c_in)
+        x_in = torch.empty((N, d), device=dev, dtype=bf)
+        ms = timed(lambda: L.mhc_route_mix(L.MHC_MIX, X, F, c_in, w_r, b_r, X, x_in, None, c_out, N, d, 1e-6, 20,
+                                           L.BF16), a.warmup, a.iters)
+        res.update(shape=[N, d], ms=ms, gbs=N * (2 * 6 * d + 64) / ms / 1e6)
+    assert L.device_error() == 0
+    print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()
