@@ -257,6 +257,7 @@ size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
 }
 
 int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace) {
+  if (Tq >= 16) return 1;
   return has_workspace && attn_splits(B, Tq, Tkv, Hkv) > 1 ? 2 : 1;
 }
 
@@ -289,6 +290,12 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
                      cudaStream_t s) {
   if (B == 0 || Tq == 0) return cudaSuccess;
+  // multi-token queries (prefill) go to the tensor-core kernel; single-token decode keeps
+  // the split-K kernel, which streams the KV slab at full width
+  if (Tq >= 16 && Tkv > 0 && gqa_tc_supported(dh, dtype, q, ld_q, gate, ld_gate, k, v, kv_cap)) {
+    cudaError_t e = gqa_attn_tc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
 #define ATTN(TT, DHV) \
   return launch_attn<TT, DHV>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, workspace, s)
   if (dtype == BF16) {

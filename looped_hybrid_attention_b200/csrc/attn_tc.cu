@@ -1,0 +1,273 @@
+// Causal GQA flash attention on the 5th-generation tensor cores, head dim 256, bf16
+// ("Loop-9B engineering teardown" §三: GQA 16 q / 4 KV heads, head dim 256, output gate).
+//
+// One CTA = 128 query rows of one q head.  Warps:
+//   0     TMA: the Q tile once (4 x [128 x 64] sub-tiles), then K and V tiles of 64 keys
+//         into a 2-stage ring (3-D maps over the per-execution slab, so keys past Tkv
+//         read as zeros);
+//   1     MMA: S_j = Q K_j^T (M 128, N 64, K 256) into one of two TMEM buffers, and
+//         O += P_j V_j (M 128, N 256, K 64; V is an MN-major operand) into TMEM;
+//   2..5  softmax, one thread per query row (TMEM lane = row, so the row max and
+//         sum are thread-local): scores -> exp2 -> bf16 P written to shared memory in
+//         the 128-byte-swizzled K-major layout the MMA reads; O is rescaled in TMEM
+//         only when the running max grows by more than 2^8 (the stale max cancels in
+//         the final O / l); finally O / l * sigmoid(gate) is stored.
+// Q K^T of tile j+1 overlaps the softmax of tile j.  All waits are bounded.
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace lk {
+namespace tc {
+
+constexpr int AT_M = 128, AT_N = 64, AT_D = 256;
+constexpr int Q_BYTES = AT_M * AT_D * 2;         // 64 KiB
+constexpr int KV_TILE = AT_N * AT_D * 2;         // 32 KiB each for K and V
+constexpr int P_BYTES = AT_M * AT_N * 2;         // 16 KiB
+constexpr int AT_SMEM = Q_BYTES + 2 * 2 * KV_TILE + P_BYTES + 1024 + 256;
+constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units
+
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tK,
+                   const __grid_constant__ CUtensorMap tV, const __nv_bfloat16* __restrict__ gate, int ld_gate,
+                   __nv_bfloat16* __restrict__ out, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
+                   float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + Q_BYTES;                      // stage s: K at s*2*KV_TILE, V at +KV_TILE
+  uint8_t* sP = sKV + 4 * KV_TILE;
+  uint64_t* bars = (uint64_t*)(sP + P_BYTES);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 12);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (3 + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (5 + b); };
+  auto s_free = [&](int b) { return bar0 + 8u * (7 + b); };
+  const uint32_t p_full = bar0 + 8u * 9, pv_done = bar0 + 8u * 10;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = gridDim.x;
+  const int qt = n_qt - 1 - blockIdx.x;               // longest causal rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (Hq / Hkv);
+  const int q0 = qt * AT_M;
+  int k_end = Tkv;
+  if (causal) k_end = min(k_end, q_off + q0 + AT_M);
+  const int n_kv = (k_end + AT_N - 1) / AT_N;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(s_free(s), 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tQ) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tK) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tV) : "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem + 256;                     // O: columns 256..511; S buffers: 0..63, 64..127
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(q_full, Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tma_load_3d(smem_u32(sQ + c * (Q_BYTES / 4)), &tQ, q_full, h * AT_D + c * 64, q0, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(kv_empty(s), ((j >> 1) & 1) ^ 1, abort_flag)) goto done;
+        mbar_expect_tx(kv_full(s), 2 * KV_TILE);
+        const uint32_t kd = smem_u32(sKV + s * 2 * KV_TILE), vd = kd + KV_TILE;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tma_load_3d(kd + c * (KV_TILE / 4), &tK, kv_full(s), c * 64, j * AT_N, b * Hkv + kvh);
+          tma_load_3d(vd + c * (KV_TILE / 4), &tV, kv_full(s), c * 64, j * AT_N, b * Hkv + kvh);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(AT_M, AT_N);
+      constexpr uint32_t id_pv = idesc_bf16(AT_M, AT_D, 1);
+      if (!mbar_wait(q_full, 0, abort_flag)) goto done;
+      const uint32_t qa = smem_u32(sQ);
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(kv_full(s), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(s_free(s), ((j >> 1) & 1) ^ 1, abort_flag)) return false;
+        fence_after();
+        const uint32_t ka = smem_u32(sKV + s * 2 * KV_TILE);
+#pragma unroll
+        for (int ks = 0; ks < AT_D / 16; ++ks) {
+          const uint32_t sub = ks >> 2, in = (ks & 3) * 32;   // 64-wide sub-tile, 16-element step
+          mma_bf16(tmem + s * AT_N, sw128_desc(qa + sub * (Q_BYTES / 4) + in), sw128_desc(ka + sub * (KV_TILE / 4) + in),
+                   id_qk, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full(s));
+        return true;
+      };
+      if (n_kv > 0 && !issue_qk(0)) goto done;
+      for (int j = 0; j < n_kv; ++j) {
+        if (j + 1 < n_kv && !issue_qk(j + 1)) goto done;
+        if (!mbar_wait(p_full, j & 1, abort_flag)) goto done;
+        fence_after();
+        const uint32_t pa = smem_u32(sP);
+        const uint32_t va = smem_u32(sKV + (j & 1) * 2 * KV_TILE + KV_TILE);
+#pragma unroll
+        for (int ks = 0; ks < AT_N / 16; ++ks)
+          mma_bf16(tO, sw128_desc(pa + ks * 32), sw128_desc_mn(va + ks * 2048, KV_TILE / 4), id_pv,
+                   (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(pv_done);
+        mma_commit(kv_empty(j & 1));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                // query row within the tile
+    const int qpos = q_off + q0 + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait(s_full(s), (j >> 1) & 1, abort_flag)) goto done;
+      fence_after();
+      uint32_t sa[32], sb[32];
+      tmem_ld32(tmem + lane_off + s * AT_N, sa);
+      tmem_ld32(tmem + lane_off + s * AT_N + 32, sb);
+      tmem_wait_ld();
+      fence_before();
+      mbar_arrive(s_free(s));
+      float t[64];
+      float mt = -INFINITY;
+      const int kbase = j * AT_N;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float raw = __uint_as_float(i < 32 ? sa[i] : sb[i - 32]);
+        const int key = kbase + i;
+        const bool ok = key < Tkv && (!causal || key <= qpos);
+        t[i] = ok ? raw * scale_log2 : -INFINITY;
+        mt = fmaxf(mt, t[i]);
+      }
+      if (j > 0 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag)) goto done;
+      if (mt > m_used + RESCALE_THRESHOLD) {
+        if (j > 0) {                                  // O holds tiles < j scaled by 2^-m_used
+          const float corr = exp2f(m_used - mt);
+          l *= corr;
+          fence_after();
+#pragma unroll 1
+          for (int c = 0; c < AT_D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            tmem_st32(tO + lane_off + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        m_used = mt;
+      }
+      // P row (bf16) into the swizzled [128 x 64] K-major tile: 16-byte chunk c of row r
+      // sits at chunk position c ^ (r & 7)
+      float psum = 0.f;
+      uint8_t* prow = sP + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(t[c * 8 + 2 * e] - m_used), exp2f(t[c * 8 + 2 * e + 1] - m_used));
+          const float2 back = __bfloat1622float2(pr);
+          psum += back.x + back.y;
+          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += psum;
+      fence_proxy_async();
+      fence_before();
+      mbar_arrive(p_full);
+    }
+    if (n_kv > 0 && !mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag)) goto done;
+    fence_after();
+    const int row = q0 + r;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < AT_D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + lane_off + c * 32, o);
+      tmem_wait_ld();
+      if (row < Tq) {
+        const long m = (long)b * Tq + row;
+        float v[32];
+        const __nv_bfloat16* gp = gate ? gate + m * ld_gate + (long)h * AT_D + c * 32 : nullptr;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float g8[8];
+          if (gp) load8(gp + i, g8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = __uint_as_float(o[i + e]) * inv;
+            v[i + e] = gp ? x / (1.f + __expf(-g8[e])) : x;
+          }
+        }
+        __nv_bfloat16* op = out + (m * Hq + h) * AT_D + c * 32;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) store8(op + i, v + i);
+      }
+    }
+  }
+done:
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+
+bool gqa_tc_supported(int dh, int dtype, const void* q, int ld_q, const void* gate, int ld_gate, const void* k,
+                      const void* v, int kv_cap) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  return dtype == BF16 && dh == tc::AT_D && al16(q) && al16(k) && al16(v) && (ld_q % 8 == 0) &&
+         (!gate || (al16(gate) && ld_gate % 8 == 0)) && kv_cap > 0;
+}
+
+cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate,
+                        int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
+                        cudaStream_t s) {
+  using namespace tc;
+  CUtensorMap mQ, mK, mV;
+  if (!make_map_3d(&mQ, q, (long)Hq * AT_D, Tq, B, ld_q, (long)Tq * ld_q, 64, AT_M)) return cudaErrorNotSupported;
+  if (!make_map_3d(&mK, k, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
+  if (!make_map_3d(&mV, v, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((Tq + AT_M - 1) / AT_M, Hq, B);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)AT_D);
+  attn_tc_kernel<<<grid, 192, AT_SMEM, s>>>(mQ, mK, mV, (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, Tq,
+                                            Tkv, q_off, Hq, Hkv, causal, scale_log2);
+  return cudaGetLastError();
+}
+
+}  // namespace lk

@@ -48,6 +48,12 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
 bool gqa_supported(int dh, int Hq, int Hkv);
 int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace);
+// tcgen05 flash attention (bf16, head dim 256); used for multi-token queries.
+bool gqa_tc_supported(int dh, int dtype, const void* q, int ld_q, const void* gate, int ld_gate, const void* k,
+                      const void* v, int kv_cap);
+cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate,
+                        int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
+                        cudaStream_t s);
 
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
                 const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,
