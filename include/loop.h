@@ -166,10 +166,16 @@ loop_status loop_decode_step(loop_model* m, loop_cache* c, const int32_t* tok, f
  * computed C = chunk tokens at a time (UT-transform form; exact up to rounding).
  * q, k [B, T, H, dk] dtype (already L2-normalised); v [B, T, H, dv] dtype;
  * g (log decay, <= 0), beta [B, T, H] fp32; state [B, H, dv, dk] fp32 in/out;
- * out [B, T, H, dv] dtype.  Supported: (dk, dv) in {(64,64), (128,128)}, chunk 64. */
+ * out [B, T, H, dv] dtype.  Supported: (dk, dv) in {(64,64), (128,128)}, chunk 64.
+ * workspace: device scratch of loop_gdn_workspace_bytes(B, T, H, dk, dv) bytes for the
+ * two-pass scan (every chunk's intra-chunk solve in parallel, then the sequential state
+ * pass), or NULL for a single-pass kernel that needs no scratch (slower).  Calls that
+ * share a workspace must not overlap on the GPU. */
 loop_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* out, int B, int T, int H,
-                          int dk, int dv, int chunk, float scale, int dtype, void* stream);
+                          int dk, int dv, int chunk, float scale, void* workspace, int dtype,
+                          void* stream);
+size_t loop_gdn_workspace_bytes(int B, int T, int H, int dk, int dv);
 
 /* One token of the same recurrence per sequence: q, k [B, H, dk]; v, out [B, H, dv];
  * g, beta [B, H] fp32; state [B, H, dv, dk] fp32 in/out. */

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(HERE, "libloop_b200.so")
 HEADER = os.path.join(HERE, "..", "include", "loop.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m looped_hybrid_attention_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python looped_hybrid_attention_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -76,7 +76,8 @@ _SIGS = {
     "loop_prefill": ([_P, _P, _P, _I, _I, _P, _P], _I),
     "loop_forward_hidden": ([_P, _P, _P, _P, _I, _I, _P], _I),
     "loop_decode_step": ([_P, _P, _P, _P, _P, _P], _I),
-    "gdn_chunk_fwd": ([_P] * 7 + [_I] * 6 + [_F, _I, _P], _I),
+    "gdn_chunk_fwd": ([_P] * 7 + [_I] * 6 + [_F, _P, _I, _P], _I),
+    "loop_gdn_workspace_bytes": ([_I] * 5, _Z),
     "gdn_step": ([_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
     "gdn_prep": ([_P, _I] + [_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
     "gqa_attn": ([_P, _I, _P, _P, _I, _P, _I, _P] + [_I] * 8 + [_P, _I, _P], _I),
@@ -274,11 +275,15 @@ class Cache:
 
 # ----------------------------------------------------------------------------- per-op calls
 
-def gdn_chunk_fwd(q, k, v, g, beta, state, out, scale, chunk=64, stream=None):
+def gdn_workspace_bytes(B, T, H, dk, dv):
+    return _lib.loop_gdn_workspace_bytes(B, T, H, dk, dv)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, state, out, scale, chunk=64, workspace=None, stream=None):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     check(_lib.gdn_chunk_fwd(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(state), ptr(out), B, T, H, dk, dv,
-                             chunk, scale, dtype_code(q), _stream(stream)), "gdn_chunk_fwd")
+                             chunk, scale, ptr(workspace), dtype_code(q), _stream(stream)), "gdn_chunk_fwd")
 
 
 def gdn_step(q, k, v, g, beta, state, out, scale, stream=None):

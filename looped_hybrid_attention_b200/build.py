@@ -2,7 +2,8 @@
 
 Each .cu file in csrc/ is compiled with relocatable device code (the kernels
 share one device error word) and linked into one shared library next to this
-file.  Usage: python -m looped_hybrid_attention_b200.build [--force] [-j N]
+file.  Usage: python looped_hybrid_attention_b200/build.py [--force] [-j N]
+(run it as a script: importing the package loads the library it builds).
 """
 from __future__ import annotations
 

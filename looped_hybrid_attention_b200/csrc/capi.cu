@@ -216,16 +216,22 @@ loop_status loop_decode_step(loop_model* m, loop_cache* c, const int32_t* tok, f
 }
 
 // ------------------------------------------------------------------ per-op entry points
+size_t loop_gdn_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
+  return gdn_workspace_bytes(B, T, H, dk, dv);
+}
+
 loop_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           float* state, void* out, int B, int T, int H, int dk, int dv, int chunk, float scale,
-                          int dtype, void* stream) {
+                          void* workspace, int dtype, void* stream) {
   REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
   REQUIRE(B >= 0 && T >= 0 && H > 0, LOOP_ERR_INVALID_ARG, "negative size");
   if (B == 0 || T == 0) return LOOP_OK;
   REQUIRE(q && k && v && g && beta && state && out, LOOP_ERR_INVALID_ARG, "NULL argument");
   REQUIRE(chunk == 64, LOOP_ERR_UNSUPPORTED, "chunk must be 64");
   REQUIRE(gdn_supported(dk, dv), LOOP_ERR_UNSUPPORTED, "(dk, dv) must be (64, 64) or (128, 128)");
-  return launched(gdn_chunk(q, k, v, g, beta, state, out, B, T, H, dk, dv, scale, dtype, S(stream)), "gdn_chunk_fwd");
+  return launched(gdn_chunk(q, k, v, g, beta, state, out, B, T, H, dk, dv, scale, dtype, S(stream), workspace),
+                  "gdn_chunk_fwd");
 }
 
 loop_status gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,

@@ -233,6 +233,345 @@ __global__ void __launch_bounds__(256) gdn_chunk_kernel(const T* __restrict__ q,
   for (int idx = tid; idx < DVS * DK; idx += nth) Sg[idx] = Ss[(idx / DK) * KP + idx % DK];
 }
 
+// ------------------------------------------------------------------ two-pass chunked scan
+// Pass 1 (gdn_intra_kernel, every chunk in parallel): cumulative log decay G, the
+// strictly lower A and the causal P = (q.k) exp(G_r - G_s), and the solve
+// (I + A) [W | U'] = [beta*gamma*K | beta*V] -- one thread per right-hand-side column,
+// the column held in registers.  Written to the workspace: W [64, dk], U' [64, dv],
+// P [64, 64], G [64] (fp32) per (b, h, chunk).
+// Pass 2 (gdn_scan_kernel, chunks in order per (b, h, dv-slice)): U = U' - W S^T,
+// O = scale (gamma Q S^T + P U), S <- exp(G_last) S + U^T (exp(G_last - G) K).  The next
+// chunk's operands are prefetched with cp.async while the current one is processed.
+template <int DK, int DV>
+struct GdnWs {
+  static constexpr int W_OFF = 0, U_OFF = GDN_C * DK, P_OFF = U_OFF + GDN_C * DV, G_OFF = P_OFF + GDN_C * GDN_C;
+  static constexpr int FLOATS = G_OFF + GDN_C;
+};
+
+size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  const long chunks = (T + GDN_C - 1) / GDN_C;
+  return (size_t)B * H * chunks * (GDN_C * (dk + dv) + GDN_C * GDN_C + GDN_C) * sizeof(float);
+}
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                        const T* __restrict__ v, const float* __restrict__ g,
+                                                        const float* __restrict__ beta, float* __restrict__ ws,
+                                                        int T_len, int H, int n_chunks) {
+  constexpr int C = GDN_C, CP = GDN_C + 4;
+  using WL = GdnWs<DK, DV>;
+  extern __shared__ float sm[];
+  float* Kt = sm;                 // [DK][CP] keys, transposed
+  float* Qt = Kt + DK * CP;       // [DK][CP] queries, transposed
+  float* As = Qt + DK * CP;       // [C][CP] strictly lower A
+  float* Gs = As + C * CP;        // [C]
+  float* Bs = Gs + C;             // [C]
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int c0 = c * C, n = min(C, T_len - c0);
+  float* blk = ws + (((long)b * H + h) * n_chunks + c) * WL::FLOATS;
+  for (int idx = tid; idx < C * DK; idx += 256) {
+    const int r = idx / DK, j = idx % DK;
+    float kv = 0.f, qv = 0.f;
+    if (r < n) {
+      const long base = (((long)b * T_len + c0 + r) * H + h) * DK + j;
+      kv = ldf(k + base);
+      qv = ldf(q + base);
+    }
+    Kt[j * CP + r] = kv;
+    Qt[j * CP + r] = qv;
+  }
+  if (tid < C) {
+    const long gi = ((long)b * T_len + c0 + tid) * H + h;
+    Gs[tid] = tid < n ? g[gi] : 0.f;
+    Bs[tid] = tid < n ? beta[gi] : 0.f;
+  }
+  __syncthreads();
+  if (tid < 32) {                 // inclusive prefix sum of the log decays
+    float a0 = Gs[2 * tid], a1 = a0 + Gs[2 * tid + 1];
+    float x = a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (tid >= o) x += y;
+    }
+    Gs[2 * tid] = x - a1 + a0;
+    Gs[2 * tid + 1] = x;
+  }
+  __syncthreads();
+  if (tid < C) blk[WL::G_OFF + tid] = Gs[tid];
+  {
+    // 4 x 4 blocks of K K^T and Q K^T on and below the diagonal
+    const int r0 = (tid >> 4) * 4, s0 = (tid & 15) * 4;
+    float ak[4][4], aq[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ak[a][e] = aq[a][e] = 0.f;
+    if (s0 <= r0 + 3) {
+#pragma unroll 4
+      for (int j = 0; j < DK; ++j) {
+        const float4 kr = *reinterpret_cast<const float4*>(Kt + j * CP + r0);
+        const float4 qr = *reinterpret_cast<const float4*>(Qt + j * CP + r0);
+        const float4 ks = *reinterpret_cast<const float4*>(Kt + j * CP + s0);
+        const float krv[4] = {kr.x, kr.y, kr.z, kr.w}, qrv[4] = {qr.x, qr.y, qr.z, qr.w};
+        const float ksv[4] = {ks.x, ks.y, ks.z, ks.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            ak[a][e] = fmaf(krv[a], ksv[e], ak[a][e]);
+            aq[a][e] = fmaf(qrv[a], ksv[e], aq[a][e]);
+          }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = r0 + a;
+      float av[4], pv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int s2 = s0 + e;
+        const float dec = s2 <= r ? expf(Gs[r] - Gs[s2]) : 0.f;
+        av[e] = s2 < r ? Bs[r] * dec * ak[a][e] : 0.f;
+        pv[e] = aq[a][e] * dec;
+      }
+      *reinterpret_cast<float4*>(As + r * CP + s0) = make_float4(av[0], av[1], av[2], av[3]);
+      *reinterpret_cast<float4*>(blk + WL::P_OFF + r * C + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+    }
+  }
+  __syncthreads();
+  if (tid < DK + DV) {
+    const int j = tid;
+    float x[C];
+    if (j < DK) {
+#pragma unroll
+      for (int r = 0; r < C; ++r) x[r] = Bs[r] * expf(Gs[r]) * Kt[j * CP + r];
+    } else {
+#pragma unroll
+      for (int r = 0; r < C; ++r)
+        x[r] = r < n ? Bs[r] * ldf(v + (((long)b * T_len + c0 + r) * H + h) * DV + (j - DK)) : 0.f;
+    }
+    // forward substitution with the unit lower-triangular I + A (A[r][s] = 0 for s >= r)
+#pragma unroll
+    for (int r = 1; r < C; ++r) {
+      float acc = x[r];
+#pragma unroll
+      for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
+        const float4 a = *reinterpret_cast<const float4*>(As + r * CP + 4 * s4);
+        acc = fmaf(-a.x, x[4 * s4], acc);
+        acc = fmaf(-a.y, x[4 * s4 + 1], acc);
+        acc = fmaf(-a.z, x[4 * s4 + 2], acc);
+        acc = fmaf(-a.w, x[4 * s4 + 3], acc);
+      }
+      x[r] = acc;
+    }
+    float* dst = j < DK ? blk + WL::W_OFF + j : blk + WL::U_OFF + (j - DK);
+    const int stride = j < DK ? DK : DV;
+#pragma unroll
+    for (int r = 0; r < C; ++r) dst[r * stride] = x[r];
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
+  const int sz = valid ? 16 : 0;                       // 0: fill zeros, read nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename T, int DK, int DV, int DVS>
+struct ScanSmem {
+  static constexpr int WP = DK + 4;                    // fp32 row pitch of W
+  static constexpr int PP = GDN_C + 4;                 // fp32 row pitch of P
+  static constexpr int QP = DK + 16 / sizeof(T);       // row pitch of Q and K (elements of T)
+  static constexpr int W_B = GDN_C * WP * 4, P_B = GDN_C * PP * 4, UP_B = GDN_C * DVS * 4,
+                       Q_B = GDN_C * QP * sizeof(T), G_B = GDN_C * 4;
+  static constexpr int BUF = W_B + P_B + UP_B + 2 * Q_B + G_B;
+  static constexpr int ST_B = DK * DVS * 4;
+  static constexpr int NBUF = (2 * BUF + 2 * ST_B + UP_B + 3 * GDN_C * 4 + 64) <= 225 * 1024 ? 2 : 1;
+  static constexpr size_t BYTES = (size_t)NBUF * BUF + 2 * ST_B + UP_B + 3 * GDN_C * 4 + 64;
+};
+
+template <typename T, int DK, int DV, int DVS>
+__global__ void __launch_bounds__(256) gdn_scan_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                       const float* __restrict__ ws, float* __restrict__ state,
+                                                       T* __restrict__ out, int T_len, int H, int n_chunks, float scale) {
+  constexpr int C = GDN_C;
+  using L = ScanSmem<T, DK, DV, DVS>;
+  using WL = GdnWs<DK, DV>;
+  constexpr int NBUF = L::NBUF;
+  extern __shared__ __align__(16) uint8_t smb[];
+  float* St[2] = {(float*)(smb + NBUF * L::BUF), (float*)(smb + NBUF * L::BUF + L::ST_B)};   // [DK][DVS]
+  float* Us = (float*)(smb + NBUF * L::BUF + 2 * L::ST_B);                                     // [C][DVS]
+  float* gam = Us + C * DVS;                                                                     // exp(G_r)
+  float* ex = gam + C;                                                                           // exp(G_last - G_s)
+  const int tid = threadIdx.x;
+  const int i0 = blockIdx.x * DVS, h = blockIdx.y, b = blockIdx.z;
+  float* Sg = state + (((long)b * H + h) * DV + i0) * DK;
+  for (int idx = tid; idx < DVS * DK; idx += 256) St[0][(idx % DK) * DVS + idx / DK] = Sg[idx];
+
+  auto buf_ptr = [&](int bi) { return smb + bi * L::BUF; };
+  auto issue = [&](int c, int bi) {
+    uint8_t* base = buf_ptr(bi);
+    float* Ws = (float*)base;
+    float* Ps = (float*)(base + L::W_B);
+    float* Ups = (float*)(base + L::W_B + L::P_B);
+    T* Qs = (T*)(base + L::W_B + L::P_B + L::UP_B);
+    T* Ks = (T*)(base + L::W_B + L::P_B + L::UP_B + L::Q_B);
+    float* Gs = (float*)(base + L::W_B + L::P_B + L::UP_B + 2 * L::Q_B);
+    const float* blk = ws + (((long)b * H + h) * n_chunks + c) * WL::FLOATS;
+    const int c0 = c * C, n = min(C, T_len - c0);
+    for (int idx = tid; idx < C * DK / 4; idx += 256) {
+      const int r = idx / (DK / 4), p = idx % (DK / 4);
+      cp_async16(Ws + r * L::WP + 4 * p, blk + WL::W_OFF + r * DK + 4 * p, true);
+    }
+    for (int idx = tid; idx < C * C / 4; idx += 256) {
+      const int r = idx / (C / 4), p = idx % (C / 4);
+      cp_async16(Ps + r * L::PP + 4 * p, blk + WL::P_OFF + r * C + 4 * p, true);
+    }
+    for (int idx = tid; idx < C * DVS / 4; idx += 256) {
+      const int r = idx / (DVS / 4), p = idx % (DVS / 4);
+      cp_async16(Ups + r * DVS + 4 * p, blk + WL::U_OFF + r * DV + i0 + 4 * p, true);
+    }
+    constexpr int PER_ROW = DK * (int)sizeof(T) / 16;
+    for (int idx = tid; idx < C * PER_ROW; idx += 256) {
+      const int r = idx / PER_ROW, p = idx % PER_ROW;
+      const bool ok = r < n;
+      const long row = (((long)b * T_len + c0 + (ok ? r : 0)) * H + h) * DK;
+      cp_async16((uint8_t*)(Qs + r * L::QP) + 16 * p, (const uint8_t*)(q + row) + 16 * p, ok);
+      cp_async16((uint8_t*)(Ks + r * L::QP) + 16 * p, (const uint8_t*)(k + row) + 16 * p, ok);
+    }
+    if (tid < C / 4) cp_async16(Gs + 4 * tid, blk + WL::G_OFF + 4 * tid, true);
+    cp_async_commit();
+  };
+
+  issue(0, 0);
+  int cur = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int bi = NBUF == 2 ? (c & 1) : 0;
+    if (NBUF == 2 && c + 1 < n_chunks) {
+      issue(c + 1, (c + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    uint8_t* base = buf_ptr(bi);
+    const float* Ws = (const float*)base;
+    const float* Ps = (const float*)(base + L::W_B);
+    const float* Ups = (const float*)(base + L::W_B + L::P_B);
+    const T* Qs = (const T*)(base + L::W_B + L::P_B + L::UP_B);
+    const T* Ks = (const T*)(base + L::W_B + L::P_B + L::UP_B + L::Q_B);
+    const float* Gs = (const float*)(base + L::W_B + L::P_B + L::UP_B + 2 * L::Q_B);
+    const float* S0 = St[cur];
+    float* S1 = St[cur ^ 1];
+    const int c0 = c * C, n = min(C, T_len - c0);
+    if (tid < C) {
+      gam[tid] = expf(Gs[tid]);
+      ex[tid] = expf(Gs[C - 1] - Gs[tid]);
+    }
+    // U = U' - W S^T : thread (r, 4 consecutive i)
+    const int r = tid >> 2, ib = (tid & 3) * 4;
+    for (int it = 0; it < DVS / 16; ++it) {
+      const int i = ib + it * 16;
+      float4 acc = *reinterpret_cast<const float4*>(Ups + r * DVS + i);
+#pragma unroll 8
+      for (int kk = 0; kk < DK; ++kk) {
+        const float w = Ws[r * L::WP + kk];
+        const float4 sv = *reinterpret_cast<const float4*>(S0 + kk * DVS + i);
+        acc.x = fmaf(-w, sv.x, acc.x);
+        acc.y = fmaf(-w, sv.y, acc.y);
+        acc.z = fmaf(-w, sv.z, acc.z);
+        acc.w = fmaf(-w, sv.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(Us + r * DVS + i) = acc;
+    }
+    __syncthreads();
+    // O = scale (gamma Q S^T + P U)
+    for (int it = 0; it < DVS / 16; ++it) {
+      const int i = ib + it * 16;
+      float4 a1 = make_float4(0, 0, 0, 0), a2 = make_float4(0, 0, 0, 0);
+#pragma unroll 8
+      for (int kk = 0; kk < DK; ++kk) {
+        const float qv = ldf(Qs + r * L::QP + kk);
+        const float4 sv = *reinterpret_cast<const float4*>(S0 + kk * DVS + i);
+        a1.x = fmaf(qv, sv.x, a1.x);
+        a1.y = fmaf(qv, sv.y, a1.y);
+        a1.z = fmaf(qv, sv.z, a1.z);
+        a1.w = fmaf(qv, sv.w, a1.w);
+      }
+      for (int s2 = 0; s2 <= r; ++s2) {
+        const float pv = Ps[r * L::PP + s2];
+        const float4 uv = *reinterpret_cast<const float4*>(Us + s2 * DVS + i);
+        a2.x = fmaf(pv, uv.x, a2.x);
+        a2.y = fmaf(pv, uv.y, a2.y);
+        a2.z = fmaf(pv, uv.z, a2.z);
+        a2.w = fmaf(pv, uv.w, a2.w);
+      }
+      if (r < n) {
+        const float gr = gam[r];
+        T* op = out + (((long)b * T_len + c0 + r) * H + h) * DV + i0 + i;
+        stf(op + 0, scale * fmaf(gr, a1.x, a2.x));
+        stf(op + 1, scale * fmaf(gr, a1.y, a2.y));
+        stf(op + 2, scale * fmaf(gr, a1.z, a2.z));
+        stf(op + 3, scale * fmaf(gr, a1.w, a2.w));
+      }
+    }
+    // S1 = exp(G_last) S0 + U^T (exp(G_last - G) K) : thread (kk, 4 consecutive i)
+    const float gl = expf(Gs[C - 1]);
+    for (int idx = tid; idx < DK * (DVS / 4); idx += 256) {
+      const int kk = idx % DK, i = (idx / DK) * 4;
+      float4 acc = *reinterpret_cast<const float4*>(S0 + kk * DVS + i);
+      acc.x *= gl;
+      acc.y *= gl;
+      acc.z *= gl;
+      acc.w *= gl;
+#pragma unroll 8
+      for (int s2 = 0; s2 < C; ++s2) {
+        const float kv = ex[s2] * ldf(Ks + s2 * L::QP + kk);
+        const float4 uv = *reinterpret_cast<const float4*>(Us + s2 * DVS + i);
+        acc.x = fmaf(uv.x, kv, acc.x);
+        acc.y = fmaf(uv.y, kv, acc.y);
+        acc.z = fmaf(uv.z, kv, acc.z);
+        acc.w = fmaf(uv.w, kv, acc.w);
+      }
+      *reinterpret_cast<float4*>(S1 + kk * DVS + i) = acc;
+    }
+    __syncthreads();
+    cur ^= 1;
+    if (NBUF == 1 && c + 1 < n_chunks) issue(c + 1, 0);
+  }
+  for (int idx = tid; idx < DVS * DK; idx += 256) Sg[idx] = St[cur][(idx % DK) * DVS + idx / DK];
+}
+
+template <typename T, int DK, int DV>
+static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                   float* state, void* out, int B, int T_len, int H, float scale, void* workspace,
+                                   cudaStream_t s) {
+  constexpr int DVS = 16;
+  const int n_chunks = (T_len + GDN_C - 1) / GDN_C;
+  const size_t smem1 = (size_t)(2 * DK * (GDN_C + 4) + GDN_C * (GDN_C + 4) + 2 * GDN_C) * sizeof(float);
+  auto k1 = gdn_intra_kernel<T, DK, DV>;
+  auto k2 = gdn_scan_kernel<T, DK, DV, DVS>;
+  using L = ScanSmem<T, DK, DV, DVS>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k1<<<dim3(n_chunks, H, B), 256, smem1, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, (float*)workspace, T_len,
+                                               H, n_chunks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,
+                                                  T_len, H, n_chunks, scale);
+  return cudaGetLastError();
+}
+
 bool gdn_supported(int dk, int dv) { return (dk == 64 && dv == 64) || (dk == 128 && dv == 128); }
 
 template <typename T, int DK, int DVS>
@@ -251,8 +590,19 @@ static cudaError_t launch_chunk(const void* q, const void* k, const void* v, con
 
 cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* state, void* out, int B, int T, int H, int dk,
-                      int dv, float scale, int dtype, cudaStream_t s) {
+                      int dv, float scale, int dtype, cudaStream_t s, void* workspace) {
   if (T == 0 || B == 0) return cudaSuccess;
+  if (workspace) {
+    if (dk == 128 && dv == 128)
+      return dtype == BF16
+                 ? launch_two_pass<__nv_bfloat16, 128, 128>(q, k, v, g, beta, state, out, B, T, H, scale, workspace, s)
+                 : launch_two_pass<float, 128, 128>(q, k, v, g, beta, state, out, B, T, H, scale, workspace, s);
+    if (dk == 64 && dv == 64)
+      return dtype == BF16
+                 ? launch_two_pass<__nv_bfloat16, 64, 64>(q, k, v, g, beta, state, out, B, T, H, scale, workspace, s)
+                 : launch_two_pass<float, 64, 64>(q, k, v, g, beta, state, out, B, T, H, scale, workspace, s);
+    return cudaErrorNotSupported;
+  }
   if (dk == 128 && dv == 128)
     return dtype == BF16 ? launch_chunk<__nv_bfloat16, 128, 16>(q, k, v, g, beta, state, out, B, T, H, dv, scale, s)
                          : launch_chunk<float, 128, 16>(q, k, v, g, beta, state, out, B, T, H, dv, scale, s);

@@ -29,9 +29,12 @@ cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, c
 cudaError_t gdn_prep(const void* P, int ld_p, const float* a_bias, const float* b_bias, void* q,
                      void* k, void* v, float* g, float* beta, int M, int H, int dk, int dv,
                      float eps, int dtype, cudaStream_t s);
+// workspace: gdn_workspace_bytes(...) of device scratch for the two-pass scan, or NULL
+// for the single-pass kernel (no scratch, slower).
 cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* state, void* out, int B, int T, int H, int dk,
-                      int dv, float scale, int dtype, cudaStream_t s);
+                      int dv, float scale, int dtype, cudaStream_t s, void* workspace = nullptr);
+size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      float* state, void* out, int B, int H, int dk, int dv, float scale, int dtype,
                      cudaStream_t s);

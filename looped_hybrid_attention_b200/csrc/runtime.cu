@@ -127,6 +127,7 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->F, M * d * es},
       {&m->coeffs, M * 8 * sizeof(float)},
       {&m->attn_ws, gqa_workspace_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_head_dim)},
+      {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
       {&m->last, (size_t)B * d * es},
   };
   for (auto& n : need) {
@@ -182,9 +183,9 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
       // flops of the chunked form per 64-token chunk and head (A and P, substitution, U, O, state)
       const double C = 64.0, chunks = (double)B * H * ((T + 63) / 64);
       const double per_chunk = 2.0 * C * C * dk + C * C * (dk + dv) + 2.0 * C * dk * dv * 3 + C * C * dv;
-      CK(prof(m, s, P_GDN_CHUNK, 1, chunks * per_chunk, io_bytes + st_bytes,
+      CK(prof(m, s, P_GDN_CHUNK, 2, chunks * per_chunk, io_bytes + st_bytes,
               [&] { return gdn_chunk(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, T, H,
-                                     dk, dv, scale, dt, s); }),
+                                     dk, dv, scale, dt, s, m->gdn_ws.p); }),
          "GDN chunked scan");
     }
     gemm_work(M, d, H * dv, EPI_STORE, m->esize, fl, by);

@@ -67,7 +67,8 @@ def main():
         beta = torch.sigmoid(torch.randn(B, T, H, device=dev, generator=g))
         S = torch.zeros(B, H, dk, dk, device=dev)
         out = torch.empty_like(v)
-        ms = timed(lambda: L.gdn_chunk_fwd(q, k, v, gg, beta, S, out, dk ** -0.5), a.warmup, a.iters)
+        ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=dev)
+        ms = timed(lambda: L.gdn_chunk_fwd(q, k, v, gg, beta, S, out, dk ** -0.5, workspace=ws), a.warmup, a.iters)
         byts = B * T * H * (4 * dk * 2 + 8) + 8 * B * H * dk * dk
         res.update(shape=[B, T, H, dk], ms=ms, gbs=byts / ms / 1e6)
     elif a.op == "attn":

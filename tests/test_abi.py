@@ -72,9 +72,9 @@ def test_model_create_validates_without_gpu():
 def test_per_op_argument_errors_without_gpu():
     P = ctypes.c_void_p(0x1000)
     # unsupported head size -> UNSUPPORTED, nothing launched
-    st = L._lib.gdn_chunk_fwd(P, P, P, P, P, P, P, 1, 64, 2, 96, 96, 64, 1.0, 1, None)
+    st = L._lib.gdn_chunk_fwd(P, P, P, P, P, P, P, 1, 64, 2, 96, 96, 64, 1.0, None, 1, None)
     assert st == 7
-    st = L._lib.gdn_chunk_fwd(P, P, P, P, P, P, P, 1, 64, 2, 128, 128, 32, 1.0, 1, None)
+    st = L._lib.gdn_chunk_fwd(P, P, P, P, P, P, P, 1, 64, 2, 128, 128, 32, 1.0, None, 1, None)
     assert st == 7 and "chunk" in L.last_error()
     st = L._lib.gqa_attn(P, 4096, P, P, 10, None, 0, P, 1, 20, 10, 0, 16, 4, 256, 1, None, 1, None)
     assert st == 2                                       # kv_cap < Tkv ... causal overrun -> SHAPE

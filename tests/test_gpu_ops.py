@@ -172,15 +172,17 @@ def _gdn_inputs(B, T, H, dk, dv, dtype, seed):
         torch.tensor(beta, dtype=torch.float32).cuda(), S0.cuda()
 
 
+@pytest.mark.parametrize("two_pass", [False, True])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("B,T,H,dk", [(2, 150, 3, 64), (1, 64, 2, 128), (1, 1, 2, 128), (2, 200, 2, 128)])
-def test_gdn_chunk_vs_recurrence(cuda, dtype, B, T, H, dk):
+def test_gdn_chunk_vs_recurrence(cuda, dtype, B, T, H, dk, two_pass):
     import looped_hybrid_attention_b200 as L
     q, k, v, g, beta, S = _gdn_inputs(B, T, H, dk, dk, dtype, seed=T + H)
     S0 = S.clone()
     out = torch.empty_like(v)
     scale = 1.0 / np.sqrt(dk)
-    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale)
+    ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=cuda) if two_pass else None
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale, workspace=ws)
     tol = TOL[dtype]
     for b in range(B):
         o_ref, S_ref = ops.gdn_recurrent(to64(q[b]), to64(k[b]), to64(v[b]), to64(g[b]), to64(beta[b]),
@@ -198,8 +200,9 @@ def test_gdn_step_and_chunk_continue(cuda, dtype):
     S0 = S.clone()
     out = torch.empty((B, T, H, dk), dtype=DT[dtype], device=cuda)
     scale = 1.0 / np.sqrt(dk)
+    ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=cuda)
     L.gdn_chunk_fwd(q[:, :T].contiguous(), k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(),
-                    beta[:, :T].contiguous(), S, out, scale)
+                    beta[:, :T].contiguous(), S, out, scale, workspace=ws)
     o_steps = []
     for t in range(T, T + 3):
         ot = torch.empty((B, H, dk), dtype=DT[dtype], device=cuda)
@@ -257,7 +260,8 @@ def test_gdn_chunk_full_length_sampled_heads(cuda):
     S0 = S.clone()
     out = torch.empty_like(v)
     scale = 1.0 / np.sqrt(dk)
-    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale)
+    ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=cuda)
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale, workspace=ws)
     for h in (0, 15):
         sl = slice(h, h + 1)
         o_ref, S_ref = ops.gdn_recurrent(to64(q[0, :, sl]), to64(k[0, :, sl]), to64(v[0, :, sl]), to64(g[0, :, sl]),
