@@ -206,6 +206,24 @@ loop_status gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype, void* stream);
 size_t loop_gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
 
+/* gqa_attn without allocation.  The pages have no counterpart to this entry point; it
+ * exists for callers that cannot allocate device memory for a workspace -- e.g. a host
+ * runtime that has given all free device memory to its own pool, or a latency-critical
+ * loop that must not take the implicit device synchronisation of cudaMalloc/cudaFree.
+ * Same arguments and result as gqa_attn (minus `workspace`); the split-K scratch is a
+ * fixed 32 MiB array in the library's device memory, held on every GPU that loads the
+ * library until the process exits.  A problem whose scratch (loop_gqa_workspace_bytes)
+ * exceeds 32 MiB is rejected with LOOP_ERR_CAPACITY and nothing is launched.  The first
+ * call on each device (with that device current) looks the array's address up with
+ * cudaGetSymbolAddress; make that first call before any stream capture.  Every call
+ * shares the array: calls that overlap on the GPU (different streams, or different host
+ * threads on one device) race on it.  The array keeps the last call's contents, but
+ * every slot a call reads is written by that call first, so nothing needs clearing.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+loop_status gqa_attn_noalloc(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                             const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv,
+                             int q_off, int Hq, int Hkv, int dh, int causal, int dtype, void* stream);
+
 /* QK-norm + partial rotary + KV write for one FA execution.  From P [M = B*T, ld_p]
  * (row blocks q | gate | k | v): q_out [M, Hq, dh] = rope(rmsnorm(q) * q_norm);
  * k = rope(rmsnorm(k) * k_norm) and v are written to the slabs k_cache, v_cache

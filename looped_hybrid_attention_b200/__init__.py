@@ -82,6 +82,7 @@ _SIGS = {
     "gdn_prep": ([_P, _I] + [_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
     "gqa_attn": ([_P, _I, _P, _P, _I, _P, _I, _P] + [_I] * 8 + [_P, _I, _P], _I),
     "loop_gqa_workspace_bytes": ([_I] * 5, _Z),
+    "gqa_attn_noalloc": ([_P, _I, _P, _P, _I, _P, _I, _P] + [_I] * 8 + [_I, _P], _I),
     "fa_prep": ([_P, _I, _P, _P, _P, _P, _P, _I] + [_I] * 7 + [_F, _F, _I, _P], _I),
     "mhc_route_mix": ([_I] + [_P] * 9 + [_I, _I, _F, _I, _I, _P], _I),
     "sinkhorn_fp32": ([_P, _P, _I, _I, _I, _P], _I),
@@ -307,6 +308,13 @@ def gqa_attn(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, H
              workspace=None, stream=None):
     check(_lib.gqa_attn(ptr(q), ld_q, ptr(k), ptr(v), kv_cap, ptr(gate), ld_gate, ptr(out), B, Tq, Tkv, q_off,
                         Hq, Hkv, dh, int(causal), ptr(workspace), dtype_code(q), _stream(stream)), "gqa_attn")
+
+
+def gqa_attn_noalloc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, dh, causal=True,
+                     stream=None):
+    """gqa_attn with the split-K scratch in the library's fixed device array (allocates nothing)."""
+    check(_lib.gqa_attn_noalloc(ptr(q), ld_q, ptr(k), ptr(v), kv_cap, ptr(gate), ld_gate, ptr(out), B, Tq, Tkv,
+                                q_off, Hq, Hkv, dh, int(causal), dtype_code(q), _stream(stream)), "gqa_attn_noalloc")
 
 
 def fa_prep(P, q_norm, k_norm, q_out, k_cache, v_cache, kv_cap, B, T, pos0, Hq, Hkv, dh, rotary_dims, rope_base,
