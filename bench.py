@@ -185,6 +185,135 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def summarize(kernels, steps, peaks, sustained=True):
+    """Roofline entry for the dominant kernel class and a per-class table."""
+    name, k = max(kernels.items(), key=lambda kv: kv[1]["ms"])
+    if k["flops"] > 0 and name in ("gemm", "attention", "gdn_chunk"):
+        achieved = k["flops"] / (k["ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s",
+                "peak_kind": ("bf16 sustained" if sustained else "bf16 burst") + " (" + peaks["source"] + ")"}
+    else:
+        achieved = k["bytes"] / (k["ms"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + peaks["source"] + ")"}
+    roof.update({"kernel": name, "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
+                 "launches": k["launches"], "ms_per_launch": round(k["ms"] / k["launches"], 4),
+                 "algorithmic_per_launch": (k["flops"] if roof["bound"] == "tensor" else k["bytes"]) / k["launches"],
+                 "traffic": None})
+    per_kernel = {}
+    total_ms = sum(v["ms"] for v in kernels.values())
+    for kname, v in sorted(kernels.items(), key=lambda kv: -kv[1]["ms"]):
+        e = {"launches": v["launches"] // steps, "ms_per_step": round(v["ms"] / steps, 3),
+             "share": round(v["ms"] / total_ms, 4)}
+        if v["flops"]:
+            e["tflops"] = round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)
+        if v["bytes"]:
+            e["gbs"] = round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)
+        per_kernel[kname] = e
+    return roof, per_kernel
+
+
+def run_decode(args, m, s, dev, world, seed):
+    """Decode at batch 64 over 32,768-token contexts (the decode configuration), greedy argmax.
+
+    By default the per-execution caches are filled with random values of the real shapes
+    (K, V ~ N(0,1) in every slab, states ~ N(0, 0.1^2)) and the cache length set to the
+    context length: the decode step's work does not depend on the cache's values.
+    --decode-real-prefill fills them with a real prefill of random ids instead.
+    """
+    import torch
+
+    import looped_hybrid_attention_b200 as L
+    import synth
+    B, ctx = args.decode_batch, args.decode_context
+    steps, warm = args.decode_steps, 3
+    c = m.cache(B, ctx + warm + 2 * steps)
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device=dev).manual_seed(seed)
+    t0 = time.time()
+    if args.decode_real_prefill:
+        ids = synth.uniform_ids((B, ctx), s.vocab, seed, "decode_ctx", device=dev)
+        lg = torch.empty((B, s.vocab), device=dev)
+        seg = 512
+        for p0 in range(0, ctx, seg):
+            m.prefill(c, ids[:, p0:p0 + seg].contiguous(), lg, stream)
+        torch.cuda.synchronize()
+    else:
+        n_fa, n_gdn = 14, 42
+        for slot in range(n_fa):
+            kp, vp = c.kv_ptrs(slot)
+            for p in (kp, vp):
+                slab = L.device_view(p, (B, s.fa_kv_heads, c.max_tokens, s.fa_head_dim), torch.bfloat16)
+                slab[:, :, :ctx].normal_(generator=g)
+        for slot in range(n_gdn):
+            st = L.device_view(c.state_ptr(slot), (B, s.gdn_heads, s.gdn_dv, s.gdn_dk), torch.float32)
+            st.normal_(generator=g).mul_(0.1)
+        c.length = ctx
+        torch.cuda.synchronize()
+    setup_s = time.time() - t0
+    tok = synth.uniform_ids((B,), s.vocab, seed, "decode_tok", device=dev)
+    nxt = torch.empty_like(tok)
+    for _ in range(warm):
+        m.decode_step(c, tok, None, nxt, stream)
+        tok, nxt = nxt, tok
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    m.profile(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        ev0.record(stream)
+        for _ in range(steps):
+            m.decode_step(c, tok, None, nxt, stream)
+            tok, nxt = nxt, tok
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    kernels = m.profile_read()
+    m.profile(False)
+    # end to end: each step's token ids come from pinned host memory and the next tokens go back
+    tok_host = tok.cpu().pin_memory()
+    nxt_host = torch.empty_like(tok_host).pin_memory()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        tok.copy_(tok_host, non_blocking=True)
+        m.decode_step(c, tok, None, nxt, stream)
+        nxt_host.copy_(nxt, non_blocking=True)
+        stream.synchronize()
+        tok_host, nxt_host = nxt_host, tok_host
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world)
+    peaks = load_peaks()
+    roof, per_kernel = summarize(kernels, steps, peaks)
+    # whole-step HBM roofline: weights per execution + KV read + GDN state read/write
+    kv_bytes, st_bytes = c.nbytes()
+    ctx_mid = ctx + warm + steps // 2
+    step_bytes = (sum(v["bytes"] for v in kernels.values()) / steps)
+    out = {"metric": "decode tokens/s (56-execution looped hybrid stack)", "workload":
+           f"9B-shape stack, decode B={B} over {ctx}-token contexts, {steps} greedy steps",
+           "value": round(B * steps * world / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms / steps, 3),
+           "context": "real prefill of random ids" if args.decode_real_prefill else
+           "random K/V and GDN states of the real shapes (decode work does not depend on cache values)",
+           "setup_s": round(setup_s, 1),
+           "e2e": {"value": round(B * steps * world / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": B * 4, "d2h_bytes_per_step": B * 4},
+           "gpu_launches": sum(v["launches"] for v in kernels.values()),
+           "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
+                             "achieved_gbs": round(step_bytes / (ms / steps / 1e3) / 1e9, 1),
+                             "peak": peaks["hbm_gbs"],
+                             "frac": round(step_bytes / (ms / steps / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+           "roofline": roof, "kernels": per_kernel, "clocks": clk.summary()}
+    del c
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -248,35 +377,9 @@ def run_ours(args, world, rank, local):
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world)
 
     peaks = load_peaks()
-    top = max(kernels.items(), key=lambda kv: kv[1]["ms"])
-    name, k = top
-    per_launch_ms = k["ms"] / k["launches"]
-    if k["flops"] > 0 and name in ("gemm", "attention", "gdn_chunk"):
-        achieved = k["flops"] / (k["ms"] / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained (" + peaks["source"] + ")"}
-    else:
-        achieved = k["bytes"] / (k["ms"] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + peaks["source"] + ")"}
-    roof.update({"kernel": name, "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
-                 "launches": k["launches"], "ms_per_launch": round(per_launch_ms, 4),
-                 "algorithmic_per_launch": (k["flops"] if roof["bound"] == "tensor" else k["bytes"]) / k["launches"],
-                 "traffic": None})
-    per_kernel = {}
-    total_ms = sum(v["ms"] for v in kernels.values())
-    for kname, v in sorted(kernels.items(), key=lambda kv: -kv[1]["ms"]):
-        e = {"launches": v["launches"] // args.steps, "ms_per_step": round(v["ms"] / args.steps, 3),
-             "share": round(v["ms"] / total_ms, 4)}
-        if v["flops"]:
-            e["tflops"] = round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)
-        if v["bytes"]:
-            e["gbs"] = round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)
-        per_kernel[kname] = e
+    roof, per_kernel = summarize(kernels, args.steps, peaks)
     launches = sum(v["launches"] for v in kernels.values())
 
-    if rank != 0:
-        return
     line = {"metric": "prefill tokens/s (56-execution looped hybrid stack)", "value": round(value, 1),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
@@ -288,6 +391,12 @@ def run_ours(args, world, rank, local):
                     "h2d_bytes_per_step": ids.numel() * 4, "d2h_bytes_per_step": logits.numel() * 4},
             "gpu_launches": launches, "roofline": roof, "kernels": per_kernel,
             "clocks": clk.summary()}
+    if not args.no_decode:
+        del c
+        torch.cuda.empty_cache()
+        line["decode"] = run_decode(args, m, s, dev, world, args.seed + rank)
+    if rank != 0:
+        return
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_entry(args.ref_tokens)
     print(json.dumps(line), flush=True)
@@ -302,6 +411,12 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-tokens", type=int, default=64, help="tokens per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--decode-batch", type=int, default=64)
+    ap.add_argument("--decode-context", type=int, default=32768)
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-real-prefill", action="store_true",
+                    help="fill the decode contexts with a real prefill instead of random cache values")
     args = ap.parse_args()
     world, rank, local = 1, int(os.environ.get("RANK", "0")), 0
     if args.impl == "ours":

@@ -136,6 +136,10 @@ loop_status loop_cache_create(const loop_model* m, int batch, int max_tokens, lo
 loop_status loop_cache_reset(loop_cache* c);          /* length 0, states zeroed (on the default stream) */
 loop_status loop_cache_destroy(loop_cache* c);
 loop_status loop_cache_length(const loop_cache* c, int* len /* host */);
+/* Declare that positions 0..len-1 of every slab and the GDN states hold a valid context
+ * written by the caller (e.g. restored from a saved cache); the next prefill or decode
+ * step appends at position len.  0 <= len <= max_tokens. */
+loop_status loop_cache_set_length(loop_cache* c, int len);
 loop_status loop_cache_bytes(const loop_cache* c, size_t* kv_bytes, size_t* state_bytes /* host */);
 /* Device pointers to one slab / state (for inspection and tests). */
 loop_status loop_cache_kv(const loop_cache* c, int fa_slot, void** k, void** v);

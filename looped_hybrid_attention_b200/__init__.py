@@ -70,6 +70,7 @@ _SIGS = {
     "loop_cache_reset": ([_P], _I),
     "loop_cache_destroy": ([_P], _I),
     "loop_cache_length": ([_P, ctypes.POINTER(ctypes.c_int)], _I),
+    "loop_cache_set_length": ([_P, _I], _I),
     "loop_cache_bytes": ([_P, ctypes.POINTER(_Z), ctypes.POINTER(_Z)], _I),
     "loop_cache_kv": ([_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_P)], _I),
     "loop_cache_state": ([_P, _I, ctypes.POINTER(_P)], _I),
@@ -257,6 +258,10 @@ class Cache:
         n = ctypes.c_int(0)
         check(_lib.loop_cache_length(self.handle, ctypes.byref(n)), "loop_cache_length")
         return n.value
+
+    @length.setter
+    def length(self, n):
+        check(_lib.loop_cache_set_length(self.handle, int(n)), "loop_cache_set_length")
 
     def nbytes(self):
         a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)

@@ -162,6 +162,13 @@ loop_status loop_cache_length(const loop_cache* c, int* len) {
   return LOOP_OK;
 }
 
+loop_status loop_cache_set_length(loop_cache* c, int len) {
+  REQUIRE(c, LOOP_ERR_INVALID_ARG, "cache is NULL");
+  REQUIRE(len >= 0 && len <= c->max_tokens, LOOP_ERR_CAPACITY, "length outside 0..max_tokens");
+  c->len = len;
+  return LOOP_OK;
+}
+
 loop_status loop_cache_bytes(const loop_cache* c, size_t* kv_bytes, size_t* state_bytes) {
   REQUIRE(c, LOOP_ERR_INVALID_ARG, "cache is NULL");
   const loop_model* m = c->model;
