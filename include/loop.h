@@ -264,10 +264,15 @@ loop_status sinkhorn_fp32(const float* logits, float* out, int N, int n, int ite
  *   1 ADD:    Y = X W^T + R, R [M, N] (row stride ldr) may alias Y
  *   2 SWIGLU: Y [M, N] = silu(X W^T) * (X W2^T), W2 [N, K] (the FFN's up map)
  *   3 F32:    Y [M, N] fp32
- * K must be a multiple of 8 for bf16.  */
+ * K must be a multiple of 8 for bf16.
+ * workspace: optional device scratch of loop_linear_workspace_bytes(M, N, K, epilogue)
+ * bytes (NULL = none).  With it, bf16 calls with M <= 128 split K across more CTAs
+ * (fp32 partial sums, then a reduction that applies the epilogue); calls sharing a
+ * workspace must not overlap on the GPU. */
 loop_status loop_linear(const void* X, int ldx, const void* W, const void* W2, const void* R,
-                        int ldr, void* Y, int ldy, int M, int N, int K, int epilogue, int dtype,
-                        void* stream);
+                        int ldr, void* Y, int ldy, int M, int N, int K, int epilogue,
+                        void* workspace, int dtype, void* stream);
+size_t loop_linear_workspace_bytes(int M, int N, int K, int epilogue);
 
 /* y = rmsnorm(x [+ r]) * w over rows of length d; if sum_out != NULL it receives x + r
  * (the residual sum).  x, r, sum_out, y [M, d] dtype; w [d] dtype. */

@@ -87,7 +87,8 @@ _SIGS = {
     "fa_prep": ([_P, _I, _P, _P, _P, _P, _P, _I] + [_I] * 7 + [_F, _F, _I, _P], _I),
     "mhc_route_mix": ([_I] + [_P] * 9 + [_I, _I, _F, _I, _I, _P], _I),
     "sinkhorn_fp32": ([_P, _P, _I, _I, _I, _P], _I),
-    "loop_linear": ([_P, _I, _P, _P, _P, _I, _P] + [_I] * 6 + [_P], _I),
+    "loop_linear": ([_P, _I, _P, _P, _P, _I, _P] + [_I] * 5 + [_P, _I, _P], _I),
+    "loop_linear_workspace_bytes": ([_I] * 4, _Z),
     "loop_rmsnorm": ([_P] * 5 + [_I, _I, _F, _I, _P], _I),
     "loop_embed": ([_P, _P, _P, _I, _I, _I, _I, _P], _I),
     "loop_argmax": ([_P, _P, _I, _I, _P], _I),
@@ -340,11 +341,16 @@ def sinkhorn_fp32(logits, out, iters, stream=None):
     check(_lib.sinkhorn_fp32(ptr(logits), ptr(out), N, n, iters, _stream(stream)), "sinkhorn_fp32")
 
 
-def linear(X, W, Y, epilogue=EPI_STORE, W2=None, R=None, stream=None):
+def linear_workspace_bytes(M, N, K, epilogue):
+    return _lib.loop_linear_workspace_bytes(M, N, K, epilogue)
+
+
+def linear(X, W, Y, epilogue=EPI_STORE, W2=None, R=None, workspace=None, stream=None):
     M, K = X.shape
     N = W.shape[0]
     check(_lib.loop_linear(ptr(X), X.stride(0), ptr(W), ptr(W2), ptr(R), R.stride(0) if R is not None else 0,
-                           ptr(Y), Y.stride(0), M, N, K, epilogue, dtype_code(X), _stream(stream)), "loop_linear")
+                           ptr(Y), Y.stride(0), M, N, K, epilogue, ptr(workspace), dtype_code(X), _stream(stream)),
+          "loop_linear")
 
 
 def rmsnorm(x, w, y, eps, r=None, sum_out=None, stream=None):

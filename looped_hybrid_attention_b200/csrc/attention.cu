@@ -243,11 +243,177 @@ __global__ void attn_combine_kernel(const float* __restrict__ ws, const T* __res
 
 static int attn_splits(int B, int Tq, int Tkv, int Hkv) {
   const long blocks = (long)B * Tq * Hkv;
-  int want = (int)((4L * 148 + blocks - 1) / blocks);
-  int cap = (Tkv + 511) / 512;
+  int want = (int)((8L * 148 + blocks - 1) / blocks);
+  int cap = (Tkv + 255) / 256;
   int s = want < cap ? want : cap;
   if (s > 32) s = 32;
   return s < 1 ? 1 : s;
+}
+
+
+// ------------------------------------------------------------------ single-token decode
+// One CTA per (sequence, KV head, key split); warp w = q head w of the group, so every
+// K/V tile is read from HBM once for the 4 heads that share it.  Tiles of 32 keys stream
+// through a 3-stage cp.async ring.  Scores: lane = key (K rows padded by 16 B so the
+// 32 lanes hit distinct banks); P.V: lanes over the head dim.
+constexpr int DEC_KT = 32, DEC_STAGES = 3;
+
+template <int DH>
+struct DecSmem {
+  static constexpr int KROW = DH * 2 + 16;            // padded K row (bytes)
+  static constexpr int VROW = DH * 2;
+  static constexpr int STAGE = DEC_KT * (KROW + VROW);
+  static constexpr int Q = 4 * DH * 4;                // 4 heads, fp32
+  static constexpr size_t BYTES = (size_t)DEC_STAGES * STAGE + Q;
+};
+
+__device__ __forceinline__ void cpa16(void* smem, const void* gmem, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(valid ? 16 : 0) : "memory");
+}
+
+template <int DH>
+__global__ void __launch_bounds__(128) attn_decode_kernel(const __nv_bfloat16* __restrict__ q, int ld_q,
+                                                          const __nv_bfloat16* __restrict__ kc,
+                                                          const __nv_bfloat16* __restrict__ vc, int kv_cap,
+                                                          const __nv_bfloat16* __restrict__ gate, int ld_gate,
+                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ ws,
+                                                          int Tkv, int q_off, int Hq, int Hkv, int causal,
+                                                          int n_split, int split_len, float scale) {
+  using L = DecSmem<DH>;
+  constexpr int PER = DH / 32;                          // dims per lane in P.V
+  constexpr int CH = DH / 8;                            // 16-byte chunks per row
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* qs = (float*)(sm + DEC_STAGES * L::STAGE);     // [4][DH]
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int rep = Hq / Hkv;
+  const int h = kvh * rep + w;
+  const bool head_ok = w < rep;
+  for (int i = threadIdx.x; i < 4 * DH; i += 128) {
+    const int hh = i / DH, j = i % DH;
+    qs[i] = hh < rep ? __bfloat162float(q[(long)b * ld_q + (long)(kvh * rep + hh) * DH + j]) * scale : 0.f;
+  }
+  int k_end = Tkv;
+  if (causal) k_end = min(k_end, q_off + 1);
+  const int k_begin = split * split_len;
+  k_end = min(k_end, k_begin + split_len);
+  const int n_tiles = k_end > k_begin ? (k_end - k_begin + DEC_KT - 1) / DEC_KT : 0;
+  const __nv_bfloat16* Kb = kc + ((long)b * Hkv + kvh) * kv_cap * DH;
+  const __nv_bfloat16* Vb = vc + ((long)b * Hkv + kvh) * kv_cap * DH;
+
+  auto issue = [&](int t) {
+    uint8_t* st = sm + (t % DEC_STAGES) * L::STAGE;
+    const int key0 = k_begin + t * DEC_KT;
+    for (int i = threadIdx.x; i < DEC_KT * CH; i += 128) {
+      const int r = i / CH, c = i % CH;
+      const int key = key0 + r;
+      const bool ok = key < k_end;
+      const long off = (long)(ok ? key : k_begin) * DH + c * 8;
+      cpa16(st + r * L::KROW + c * 16, Kb + off, ok);
+      cpa16(st + DEC_KT * L::KROW + r * L::VROW + c * 16, Vb + off, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+#pragma unroll
+  for (int t = 0; t < DEC_STAGES - 1; ++t) {
+    if (t < n_tiles) issue(t);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  float mx = -INFINITY, l = 0.f, o[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) o[u] = 0.f;
+  const float* qh = qs + w * DH;
+  for (int t = 0; t < n_tiles; ++t) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(DEC_STAGES - 2) : "memory");
+    __syncthreads();
+    const uint8_t* st = sm + (t % DEC_STAGES) * L::STAGE;
+    // scores: lane = key
+    const uint8_t* krow = st + lane * L::KROW;
+    float sc = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < CH; ++c) {
+      float kf[8];
+      load8(reinterpret_cast<const __nv_bfloat16*>(krow + c * 16), kf);
+      const float4 q0 = *reinterpret_cast<const float4*>(qh + c * 8);
+      const float4 q1 = *reinterpret_cast<const float4*>(qh + c * 8 + 4);
+      sc = fmaf(kf[0], q0.x, sc); sc = fmaf(kf[1], q0.y, sc); sc = fmaf(kf[2], q0.z, sc); sc = fmaf(kf[3], q0.w, sc);
+      sc = fmaf(kf[4], q1.x, sc); sc = fmaf(kf[5], q1.y, sc); sc = fmaf(kf[6], q1.z, sc); sc = fmaf(kf[7], q1.w, sc);
+    }
+    const int key = k_begin + t * DEC_KT + lane;
+    if (key >= k_end) sc = -INFINITY;
+    const float mnew = fmaxf(mx, warp_max(sc));
+    const float p = expf(sc - mnew);
+    const float corr = expf(mx - mnew);
+    l = l * corr + warp_sum(p);
+    mx = mnew;
+    // P.V: lanes over the head dim
+    const uint8_t* vt = st + DEC_KT * L::KROW;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) o[u] *= corr;
+#pragma unroll 4
+    for (int r = 0; r < DEC_KT; ++r) {
+      const float pr = __shfl_sync(0xffffffffu, p, r);
+      float vf[PER];
+      const __nv_bfloat16* vrow = reinterpret_cast<const __nv_bfloat16*>(vt + r * L::VROW) + lane * PER;
+      if (PER == 8) {
+        load8(vrow, vf);
+      } else {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) vf[u] = __bfloat162float(vrow[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < PER; ++u) o[u] = fmaf(pr, vf[u], o[u]);
+    }
+    __syncthreads();
+    if (t + DEC_STAGES - 1 < n_tiles) issue(t + DEC_STAGES - 1);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  if (!head_ok) return;
+  if (n_split == 1) {
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const __nv_bfloat16* gp = gate ? gate + (long)b * ld_gate + (long)h * DH + lane * PER : nullptr;
+    __nv_bfloat16* op = out + ((long)b * Hq + h) * DH + lane * PER;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      float r = o[u] * inv;
+      if (gp) r *= sigmoidf_acc(__bfloat162float(gp[u]));
+      op[u] = __float2bfloat16(r);
+    }
+  } else {
+    float* wp = ws + (((long)b * Hq + h) * n_split + split) * (DH + 2);
+    if (lane == 0) { wp[0] = mx; wp[1] = l; }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) wp[2 + lane * PER + u] = o[u];
+  }
+}
+
+template <int DH>
+static cudaError_t launch_decode(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate,
+                                 int ld_gate, void* out, int B, int Tkv, int q_off, int Hq, int Hkv, int causal,
+                                 void* workspace, cudaStream_t s) {
+  using L = DecSmem<DH>;
+  const int n_split = workspace ? attn_splits(B, 1, Tkv, Hkv) : 1;
+  const int split_len = (((Tkv + n_split - 1) / n_split) + DEC_KT - 1) / DEC_KT * DEC_KT;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(n_split, Hkv, B);
+  attn_decode_kernel<DH><<<grid, 128, L::BYTES, s>>>(
+      (const __nv_bfloat16*)q, ld_q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, kv_cap,
+      (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, (float*)workspace, Tkv, q_off, Hq, Hkv, causal,
+      n_split, split_len, 1.f / sqrtf((float)DH));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || n_split == 1) return e;
+  const long rows = (long)B * Hq;
+  attn_combine_kernel<__nv_bfloat16, DH><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+      (const float*)workspace, (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, rows, Hq, n_split);
+  return cudaGetLastError();
 }
 
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
@@ -295,6 +461,15 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
   if (Tq >= 16 && Tkv > 0 && gqa_tc_supported(dh, dtype, q, ld_q, gate, ld_gate, k, v, kv_cap)) {
     cudaError_t e = gqa_attn_tc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, s);
     if (e != cudaErrorNotSupported) return e;
+  }
+  // single-token decode (bf16, <= 4 q heads per KV head): the tiled flash-decode kernel
+  if (Tq == 1 && dtype == BF16 && Hq / Hkv <= 4 && (dh == 256 || dh == 128 || dh == 64) &&
+      ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0)) {
+    if (dh == 256)
+      return launch_decode<256>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
+    if (dh == 128)
+      return launch_decode<128>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
+    return launch_decode<64>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
   }
 #define ATTN(TT, DHV) \
   return launch_attn<TT, DHV>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, workspace, s)

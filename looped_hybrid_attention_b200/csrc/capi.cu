@@ -324,8 +324,13 @@ loop_status sinkhorn_fp32(const float* logits, float* out, int N, int n, int ite
   return launched(sinkhorn(logits, out, N, n, iters, S(stream)), "sinkhorn_fp32");
 }
 
+size_t loop_linear_workspace_bytes(int M, int N, int K, int epilogue) {
+  if (M <= 0 || N <= 0 || K <= 0 || epilogue < EPI_STORE || epilogue > EPI_F32) return 0;
+  return linear_workspace_bytes(M, N, K, epilogue);
+}
+
 loop_status loop_linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y,
-                        int ldy, int M, int N, int K, int epilogue, int dtype, void* stream) {
+                        int ldy, int M, int N, int K, int epilogue, void* workspace, int dtype, void* stream) {
   REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
   REQUIRE(epilogue >= EPI_STORE && epilogue <= EPI_F32, LOOP_ERR_INVALID_ARG, "epilogue must be 0..3");
   REQUIRE(M >= 0 && N >= 0 && K > 0, LOOP_ERR_INVALID_ARG, "bad size");
@@ -335,7 +340,9 @@ loop_status loop_linear(const void* X, int ldx, const void* W, const void* W2, c
   if (epilogue == EPI_ADD) REQUIRE(R && ldr >= N, LOOP_ERR_INVALID_ARG, "ADD needs R with ldr >= N");
   if (epilogue == EPI_SWIGLU) REQUIRE(W2, LOOP_ERR_INVALID_ARG, "SWIGLU needs W2");
   if (dtype == LOOP_BF16) REQUIRE(K % 8 == 0 && ldx % 8 == 0, LOOP_ERR_SHAPE, "bf16 needs K and ldx multiples of 8");
-  return launched(linear(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epilogue, dtype, S(stream)), "loop_linear");
+  const size_t ws_bytes = workspace ? linear_workspace_bytes(M, N, K, epilogue) : 0;
+  return launched(linear(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epilogue, dtype, S(stream), workspace, ws_bytes),
+                  "loop_linear");
 }
 
 loop_status loop_rmsnorm(const void* x, const void* r, void* sum_out, const void* w, void* y, int M, int d, float eps,

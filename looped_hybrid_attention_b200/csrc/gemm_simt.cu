@@ -96,9 +96,10 @@ cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, c
 }
 
 cudaError_t linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
-                   void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s) {
+                   void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s, void* ws,
+                   size_t ws_bytes) {
   if (dtype == BF16) {
-    cudaError_t e = linear_tc(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, s);
+    cudaError_t e = linear_tc(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, s, ws, ws_bytes);
     if (e != cudaErrorNotSupported) return e;
   }
   return linear_simt(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, dtype, s);

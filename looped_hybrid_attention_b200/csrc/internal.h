@@ -17,11 +17,16 @@ cudaError_t embed(const int32_t* ids, const void* E, void* out, int M, int d, in
                   cudaStream_t s);
 cudaError_t argmax(const float* logits, int32_t* next, int B, int V, cudaStream_t s);
 
+// ws / ws_bytes: optional scratch for split-K when M <= 128 (linear_workspace_bytes).
 cudaError_t linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
-                   void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s);
+                   void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s, void* ws = nullptr,
+                   size_t ws_bytes = 0);
 // tcgen05 path (bf16); returns cudaErrorNotSupported for shapes it does not take.
 cudaError_t linear_tc(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
-                      void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s);
+                      void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s, void* ws = nullptr,
+                      size_t ws_bytes = 0);
+size_t linear_workspace_bytes(int M, int N, int K, int epi);
+int linear_launches(int M, int N, int K, int epi, const void* ws, size_t ws_bytes);
 cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, const void* R,
                         int ldr, void* Y, int ldy, int M, int N, int K, int epi, int dtype,
                         cudaStream_t s);

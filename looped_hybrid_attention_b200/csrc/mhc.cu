@@ -159,10 +159,141 @@ __global__ void __launch_bounds__(128) mhc_kernel(int mode, const T* __restrict_
   }
 }
 
+// Few tokens (decode): one CTA per token, threads split the hidden dimension, and the
+// 9 routing sums are reduced across the block.
+template <typename T>
+__global__ void __launch_bounds__(512) mhc_token_kernel(int mode, const T* __restrict__ X_in, const T* __restrict__ F,
+                                                        const float* __restrict__ coeffs_in,
+                                                        const float* __restrict__ w_r, const float* __restrict__ b_r,
+                                                        T* X_out, T* __restrict__ x_in, T* __restrict__ h_out,
+                                                        float* __restrict__ coeffs_out, int d, float eps, int iters) {
+  __shared__ float red[9][16];
+  __shared__ float coef[4];
+  const long tok = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  float hp0 = 0.f, hp1 = 0.f, r00 = 0.f, r01 = 0.f, r10 = 0.f, r11 = 0.f;
+  if (mode == MHC_MIX || mode == MHC_MERGE) {
+    const float* c = coeffs_in + tok * 8;
+    hp0 = c[2]; hp1 = c[3]; r00 = c[4]; r01 = c[5]; r10 = c[6]; r11 = c[7];
+  }
+  const T* X = (mode == MHC_OPEN) ? X_in + tok * d : X_in + tok * 2 * d;
+  float l[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ss = 0.f;
+  for (int j = tid * 8; j < d; j += blockDim.x * 8) {
+    float y0[8], y1[8];
+    if (mode == MHC_OPEN) {
+      load8(X + j, y0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y1[i] = y0[i];
+    } else if (mode == MHC_ROUTE) {
+      load8(X + j, y0);
+      load8(X + d + j, y1);
+    } else {
+      float x0[8], x1[8], f[8];
+      load8(X + j, x0);
+      load8(X + d + j, x1);
+      load8(F + tok * d + j, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        y0[i] = r00 * x0[i] + r01 * x1[i] + hp0 * f[i];
+        y1[i] = r10 * x0[i] + r11 * x1[i] + hp1 * f[i];
+      }
+      if (mode == MHC_MERGE) {
+        float h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = 0.5f * (y0[i] + y1[i]);
+        store8(h_out + tok * d + j, h);
+        continue;
+      }
+      round8<T>(y0);
+      round8<T>(y1);
+    }
+    if (mode != MHC_ROUTE) {
+      store8(X_out + tok * 2 * d + j, y0);
+      store8(X_out + tok * 2 * d + d + j, y1);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ss += y0[i] * y0[i] + y1[i] * y1[i];
+      const float4* w0 = reinterpret_cast<const float4*>(w_r + (long)(j + i) * 8);
+      const float4* w1 = reinterpret_cast<const float4*>(w_r + (long)(d + j + i) * 8);
+      const float4 a0 = __ldg(w0), a1 = __ldg(w0 + 1), b0 = __ldg(w1), b1 = __ldg(w1 + 1);
+      l[0] += y0[i] * a0.x + y1[i] * b0.x;
+      l[1] += y0[i] * a0.y + y1[i] * b0.y;
+      l[2] += y0[i] * a0.z + y1[i] * b0.z;
+      l[3] += y0[i] * a0.w + y1[i] * b0.w;
+      l[4] += y0[i] * a1.x + y1[i] * b1.x;
+      l[5] += y0[i] * a1.y + y1[i] * b1.y;
+      l[6] += y0[i] * a1.z + y1[i] * b1.z;
+      l[7] += y0[i] * a1.w + y1[i] * b1.w;
+    }
+  }
+  if (mode == MHC_MERGE) return;
+  ss = warp_sum(ss);
+#pragma unroll
+  for (int o = 0; o < 8; ++o) l[o] = warp_sum(l[o]);
+  if (lane == 0) {
+    red[8][wid] = ss;
+#pragma unroll
+    for (int o = 0; o < 8; ++o) red[o][wid] = l[o];
+  }
+  __syncthreads();
+  if (wid == 0) {
+    float v[9];
+#pragma unroll
+    for (int o = 0; o < 9; ++o) v[o] = warp_sum(lane < nw ? red[o][lane] : 0.f);
+    const float inv = rsqrtf(v[8] / (float)(2 * d) + eps);
+    float lt[8];
+#pragma unroll
+    for (int o = 0; o < 8; ++o) lt[o] = v[o] * inv + b_r[o];
+    const float pre0 = sigmoidf_acc(lt[0]), pre1 = sigmoidf_acc(lt[1]);
+    float m[4];
+    const float mx = fmaxf(fmaxf(lt[4], lt[5]), fmaxf(lt[6], lt[7]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = expf(lt[4 + i] - mx);
+    sinkhorn2(m, iters);
+    if (lane == 0) {
+      float4* c = reinterpret_cast<float4*>(coeffs_out + tok * 8);
+      c[0] = make_float4(pre0, pre1, 2.f * sigmoidf_acc(lt[2]), 2.f * sigmoidf_acc(lt[3]));
+      c[1] = make_float4(m[0], m[1], m[2], m[3]);
+      coef[0] = pre0;
+      coef[1] = pre1;
+    }
+  }
+  __syncthreads();
+  const float pre0 = coef[0], pre1 = coef[1];
+  const T* Xr = (mode == MHC_ROUTE) ? X : X_out + tok * 2 * d;
+  for (int j = tid * 8; j < d; j += blockDim.x * 8) {
+    float a[8], bb[8], o[8];
+    if (mode == MHC_OPEN) {
+      load8(X + j, a);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = (pre0 + pre1) * a[i];
+    } else {
+      load8(Xr + j, a);
+      load8(Xr + d + j, bb);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = pre0 * a[i] + pre1 * bb[i];
+    }
+    store8(x_in + tok * d + j, o);
+  }
+}
+
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
                 const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,
                 int d, float eps, int iters, int dtype, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
+  if (N < 1024) {           // few tokens: spread each token over a CTA
+    const int threads = d >= 4096 ? 512 : (d >= 2048 ? 256 : 128);
+    if (dtype == BF16)
+      mhc_token_kernel<__nv_bfloat16><<<N, threads, 0, s>>>(
+          mode, (const __nv_bfloat16*)X_in, (const __nv_bfloat16*)F, coeffs_in, w_r, b_r, (__nv_bfloat16*)X_out,
+          (__nv_bfloat16*)x_in, (__nv_bfloat16*)h_out, coeffs_out, d, eps, iters);
+    else
+      mhc_token_kernel<float><<<N, threads, 0, s>>>(mode, (const float*)X_in, (const float*)F, coeffs_in, w_r, b_r,
+                                                    (float*)X_out, (float*)x_in, (float*)h_out, coeffs_out, d, eps,
+                                                    iters);
+    return cudaGetLastError();
+  }
   constexpr int TPW = 4, warps = 4;
   dim3 grid((unsigned)(((long)N + TPW * warps - 1) / (TPW * warps)));
   if (dtype == BF16)

@@ -128,6 +128,10 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->coeffs, M * 8 * sizeof(float)},
       {&m->attn_ws, gqa_workspace_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_head_dim)},
       {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
+      // split-K partials for projections with few tokens (the widest: the FFN gate/up pair)
+      {&m->gemm_ws, M <= 128 ? linear_workspace_bytes((int)M, std::max(c.ffn, std::max(m->in_fa, m->in_gdn)), c.d,
+                                                      EPI_SWIGLU)
+                             : 0},
       {&m->last, (size_t)B * d * es},
   };
   for (auto& n : need) {
@@ -155,15 +159,19 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
   const int d = cf.d, dt = cf.dtype;
   const double es = (double)m->esize;
   double fl, by;
+  // kernel launches of one projection (2 when split-K adds its reduction)
+  auto gl = [&](long Mm, int N, int K, int epi) {
+    return cf.dtype == LOOP_BF16 ? linear_launches((int)Mm, N, K, epi, m->gemm_ws.p, m->gemm_ws.bytes) : 1;
+  };
   CK(prof(m, s, P_RMSNORM, 1, 0, es * (2.0 * M * d + d),
           [&] { return rmsnorm(x, nullptr, nullptr, w.attn_norm, m->xn.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (mixer)");
   if (r.kind == 0) {
     const int H = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
     gemm_work(M, m->in_gdn, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
+    CK(prof(m, s, P_GEMM, gl(M, m->in_gdn, d, EPI_STORE), fl, by,
             [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d,
-                                EPI_STORE, dt, s); }),
+                                EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "GDN input projection");
     CK(prof(m, s, P_GDN_PREP, 1, 0, (double)M * (es * (m->in_gdn + 2.0 * H * dk + H * dv) + 8.0 * H),
             [&] { return lk::gdn_prep(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p,
@@ -189,16 +197,16 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
          "GDN chunked scan");
     }
     gemm_work(M, d, H * dv, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
+    CK(prof(m, s, P_GEMM, gl(M, d, H * dv, EPI_STORE), fl, by,
             [&] { return linear(m->o.p, H * dv, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, H * dv, EPI_STORE,
-                                dt, s); }),
+                                dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "GDN output projection");
   } else {
     const int Hq = cf.fa_q_heads, Hkv = cf.fa_kv_heads, dh = cf.fa_head_dim;
     gemm_work(M, m->in_fa, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
+    CK(prof(m, s, P_GEMM, gl(M, m->in_fa, d, EPI_STORE), fl, by,
             [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d,
-                                EPI_STORE, dt, s); }),
+                                EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "FA input projection");
     char* kbase = (char*)c->kv.p + (size_t)r.slot * 2 * c->kv_slab_elems * m->esize;
     char* vbase = kbase + c->kv_slab_elems * m->esize;
@@ -215,9 +223,9 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
                                       pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s); }),
        "GQA attention");
     gemm_work(M, d, Hq * dh, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
+    CK(prof(m, s, P_GEMM, gl(M, d, Hq * dh, EPI_STORE), fl, by,
             [&] { return linear(m->o.p, Hq * dh, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, Hq * dh,
-                                EPI_STORE, dt, s); }),
+                                EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "FA output projection");
   }
   // u = x + mix; FFN on RMSNorm(u)
@@ -225,15 +233,15 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
           [&] { return rmsnorm(x, m->mix.p, m->u.p, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (FFN)");
   gemm_work(M, cf.ffn, d, EPI_SWIGLU, m->esize, fl, by);
-  CK(prof(m, s, P_GEMM, 1, fl, by,
+  CK(prof(m, s, P_GEMM, gl(M, cf.ffn, d, EPI_SWIGLU), fl, by,
           [&] { return linear(m->un.p, d, w.w_gate, w.w_up, nullptr, 0, m->act.p, cf.ffn, (int)M, cf.ffn, d, EPI_SWIGLU,
-                              dt, s); }),
+                              dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
      "FFN gate/up (SwiGLU)");
   gemm_work(M, d, cf.ffn, EPI_ADD, m->esize, fl, by);
   const void* res = r.in_loop ? m->mix.p : m->u.p;
   void* dst = r.in_loop ? m->F.p : h_out;
-  CK(prof(m, s, P_GEMM, 1, fl, by,
-          [&] { return linear(m->act.p, cf.ffn, w.w_down, nullptr, res, d, dst, d, (int)M, d, cf.ffn, EPI_ADD, dt, s); }),
+  CK(prof(m, s, P_GEMM, gl(M, d, cf.ffn, EPI_ADD), fl, by,
+          [&] { return linear(m->act.p, cf.ffn, w.w_down, nullptr, res, d, dst, d, (int)M, d, cf.ffn, EPI_ADD, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
      "FFN down (+ residual)");
   return LOOP_OK;
 }
@@ -305,7 +313,7 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
     gemm_work(B, cf.vocab, cf.d, EPI_F32, m->esize, fl, by);
     CK(prof(m, s, P_LMHEAD, 1, fl, by,
             [&] { return linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, logits_last, cf.vocab, B, cf.vocab,
-                                cf.d, EPI_F32, cf.dtype, s); }),
+                                cf.d, EPI_F32, cf.dtype, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "LM head");
   }
   return LOOP_OK;
@@ -338,7 +346,7 @@ loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* 
   gemm_work(B, cf.vocab, cf.d, EPI_F32, m->esize, fl, by);
   CK(prof(m, s, P_LMHEAD, 1, fl, by,
           [&] { return linear(m->last.p, cf.d, m->lm_head, nullptr, nullptr, 0, lg, cf.vocab, B, cf.vocab, cf.d, EPI_F32,
-                              cf.dtype, s); }),
+                              cf.dtype, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
      "LM head");
   CK(prof(m, s, P_ARGMAX, 1, 0, 4.0 * B * cf.vocab + 4.0 * B, [&] { return argmax(lg, next, B, cf.vocab, s); }),
      "argmax");

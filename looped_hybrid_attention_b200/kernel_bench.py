@@ -4,6 +4,7 @@
   python -m looped_hybrid_attention_b200.kernel_bench gdn --T 8192 --H 16
   python -m looped_hybrid_attention_b200.kernel_bench attn --T 8192
   python -m looped_hybrid_attention_b200.kernel_bench mhc --T 8192
+  python -m looped_hybrid_attention_b200.kernel_bench decode --B 16 --T 32768
 
 Inputs are random bf16 tensors created on the device (larger than L2 at the default
 sizes); the printed rate uses the same algorithmic flop/byte counts as bench.py.
@@ -33,7 +34,7 @@ def timed(fn, warmup, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemm", "gdn", "attn", "mhc"])
+    ap.add_argument("op", choices=["gemm", "gdn", "attn", "decode", "mhc"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
@@ -80,6 +81,15 @@ def main():
                    a.warmup, a.iters)
         flops = 4.0 * Hq * dh * B * T * (T + 1) / 2
         res.update(shape=[B, T, Hq, Hkv, dh], ms=ms, tflops=flops / ms / 1e9)
+    elif a.op == "decode":
+        B, T, Hq, Hkv, dh = a.B, a.T, 16, 4, 256
+        q, gate = r(B, Hq * dh), r(B, Hq * dh)
+        K, V = r(B, Hkv, T, dh), r(B, Hkv, T, dh)
+        out = torch.empty((B, Hq * dh), device=dev, dtype=bf)
+        ws = torch.empty(L.gqa_workspace_bytes(B, 1, T, Hq, dh) // 4 + 1, device=dev)
+        ms = timed(lambda: L.gqa_attn(q, Hq * dh, K, V, T, gate, Hq * dh, out, B, 1, T, T - 1, Hq, Hkv, dh, True, ws),
+                   a.warmup, a.iters)
+        res.update(shape=[B, T, Hq, Hkv, dh], ms=ms, gbs=B * Hkv * T * dh * 2 * 2 / ms / 1e6)
     else:
         N, d = a.B * a.T, 4096
         X, F = r(N, 2, d), r(N, d)

@@ -84,5 +84,5 @@ def test_per_op_argument_errors_without_gpu():
     assert st == 1 and "F" in L.last_error()
     st = L._lib.fa_prep(P, 10240, P, P, P, P, P, 100, 1, 64, 50, 16, 4, 256, 64, 1e4, 1e-6, 1, None)
     assert st == 5                                       # positions past the slab -> CAPACITY
-    st = L._lib.loop_linear(P, 100, P, None, None, 0, P, 64, 4, 64, 100, 0, 1, None)
+    st = L._lib.loop_linear(P, 100, P, None, None, 0, P, 64, 4, 64, 100, 0, None, 1, None)
     assert st == 2                                       # bf16 needs K % 8 == 0

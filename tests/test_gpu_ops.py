@@ -34,7 +34,7 @@ def test_sinkhorn_fp32(cuda, n):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19)])
+@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19), (4096, 1501), (256, 2050)])
 def test_mhc_modes(cuda, dtype, d, N):
     import looped_hybrid_attention_b200 as L
     code = L.BF16 if dtype == "bf16" else L.F32
@@ -136,24 +136,30 @@ def test_embed_and_argmax(cuda):
 
 # ----------------------------------------------------------------------------- projections
 
+@pytest.mark.parametrize("split_k", [False, True])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("M,N,K", [(200, 300, 256), (1, 1000, 512), (130, 64, 4096)])
-def test_linear_epilogues(cuda, dtype, M, N, K):
+@pytest.mark.parametrize("M,N,K", [(200, 300, 256), (1, 1000, 512), (130, 64, 4096), (64, 4104, 2048),
+                                   (64, 1000, 12288)])
+def test_linear_epilogues(cuda, dtype, M, N, K, split_k):
     import looped_hybrid_attention_b200 as L
+    ws = None
+    if split_k:
+        nb = max(L.linear_workspace_bytes(M, N, K, e) for e in (0, 1, 2, 3))
+        ws = torch.empty(max(nb, 16) // 4, device=cuda)
     X = rnd((M, K), 12, "X", dtype=dtype)
     W = rnd((N, K), 13, "W", std=0.02, dtype=dtype)
     W2 = rnd((N, K), 14, "W2", std=0.02, dtype=dtype)
     R = rnd((M, N), 15, "R", dtype=dtype)
     Y = torch.empty((M, N), dtype=DT[dtype], device=cuda)
     ref = ops.linear(to64(X), to64(W))
-    L.linear(X, W, Y, L.EPI_STORE)
+    L.linear(X, W, Y, L.EPI_STORE, workspace=ws)
     assert rel_l2(to64(Y), ref) < TOL[dtype]
-    L.linear(X, W, Y, L.EPI_ADD, R=R)
+    L.linear(X, W, Y, L.EPI_ADD, R=R, workspace=ws)
     assert rel_l2(to64(Y), ref + to64(R)) < TOL[dtype]
-    L.linear(X, W, Y, L.EPI_SWIGLU, W2=W2)
+    L.linear(X, W, Y, L.EPI_SWIGLU, W2=W2, workspace=ws)
     assert rel_l2(to64(Y), ops.silu(ref) * ops.linear(to64(X), to64(W2))) < TOL[dtype]
     Yf = torch.empty((M, N), dtype=torch.float32, device=cuda)
-    L.linear(X, W, Yf, L.EPI_F32)
+    L.linear(X, W, Yf, L.EPI_F32, workspace=ws)
     assert rel_l2(to64(Yf), ref) < (1e-5 if dtype == "fp32" else 1e-4)
 
 
@@ -320,22 +326,26 @@ def test_fa_prep_and_attention(cuda, dtype, B, T, Hq, Hkv, dh, rot, pos0):
             assert rel_l2(to64(out.view(B, T, Hq, dh)[b]), ref) < tol
 
 
-@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_decode_attention_split_k(cuda, dtype):
+@pytest.mark.parametrize("dtype,dh,Hq,Hkv", [("fp32", 256, 16, 4), ("bf16", 256, 16, 4), ("bf16", 128, 8, 2),
+                                              ("bf16", 64, 4, 1), ("bf16", 256, 6, 2)])
+def test_decode_attention_split_k(cuda, dtype, dh, Hq, Hkv):
     """One query per sequence over a long slab: split-K partials + combine (with workspace) equal brute force."""
     import looped_hybrid_attention_b200 as L
-    B, Hq, Hkv, dh, L_ctx = 4, 16, 4, 256, 3000
+    B, L_ctx = 4, 3000
     cap = L_ctx + 10
     q = rnd((B, Hq, dh), 30, "qd", dtype=dtype)
     Kc = rnd((B, Hkv, cap, dh), 31, "Kd", dtype=dtype)
     Vc = rnd((B, Hkv, cap, dh), 32, "Vd", dtype=dtype)
+    gate = rnd((B, Hq * dh), 33, "gd", dtype=dtype)
     out = torch.empty((B, Hq * dh), dtype=DT[dtype], device=cuda)
     ws = torch.empty(L.gqa_workspace_bytes(B, 1, L_ctx, Hq, dh) // 4 + 1, device=cuda)
-    L.gqa_attn(q, Hq * dh, Kc, Vc, cap, None, 0, out, B, 1, L_ctx, L_ctx - 1, Hq, Hkv, dh, True, ws)
-    for b in range(B):
-        ref = ops.attention(to64(q[b])[None], to64(Kc[b, :, :L_ctx]).transpose(1, 0, 2),
-                            to64(Vc[b, :, :L_ctx]).transpose(1, 0, 2), [L_ctx - 1])
-        assert rel_l2(to64(out[b]).reshape(1, Hq, dh), ref) < TOL[dtype]
+    for workspace in (ws, None):                    # split-K with combine, and a single pass
+        L.gqa_attn(q, Hq * dh, Kc, Vc, cap, gate, Hq * dh, out, B, 1, L_ctx, L_ctx - 1, Hq, Hkv, dh, True, workspace)
+        for b in range(B):
+            ref = ops.attention(to64(q[b])[None], to64(Kc[b, :, :L_ctx]).transpose(1, 0, 2),
+                                to64(Vc[b, :, :L_ctx]).transpose(1, 0, 2), [L_ctx - 1])
+            ref = ref * ops.sigmoid(to64(gate[b]).reshape(1, Hq, dh))
+            assert rel_l2(to64(out[b]).reshape(1, Hq, dh), ref) < TOL[dtype]
 
 
 def test_attention_single_key_and_zero_query(cuda):
