@@ -14,6 +14,8 @@
 // Rows of S are independent, so each CTA owns DVS rows of one (b, h) and walks
 // the chunks in order; the dv split gives B*H*dv/DVS CTAs.  All decay factors are
 // exp of non-positive numbers, so nothing overflows.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -253,13 +255,22 @@ size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv) {
   return (size_t)B * H * chunks * (GDN_C * (dk + dv) + GDN_C * GDN_C + GDN_C) * sizeof(float);
 }
 
-template <typename T, int DK, int DV>
+// Workspace block of the tensor-core scan (bf16 models): W and P in bf16 (they are MMA
+// operands), U' and G in fp32.  Byte offsets within one (b, h, chunk) block.
+template <int DK, int DV>
+struct GdnWsB {
+  static constexpr int W_OFF = 0, U_OFF = GDN_C * DK * 2, P_OFF = U_OFF + GDN_C * DV * 4,
+                       G_OFF = P_OFF + GDN_C * GDN_C * 2, BYTES = G_OFF + GDN_C * 4;
+};
+
+template <typename T, int DK, int DV, bool WB>
 __global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ g,
                                                         const float* __restrict__ beta, float* __restrict__ ws,
                                                         int T_len, int H, int n_chunks) {
   constexpr int C = GDN_C, CP = GDN_C + 4;
   using WL = GdnWs<DK, DV>;
+  using WLB = GdnWsB<DK, DV>;
   extern __shared__ float sm[];
   float* Kt = sm;                 // [DK][CP] keys, transposed
   float* Qt = Kt + DK * CP;       // [DK][CP] queries, transposed
@@ -269,6 +280,7 @@ __global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q,
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int c0 = c * C, n = min(C, T_len - c0);
   float* blk = ws + (((long)b * H + h) * n_chunks + c) * WL::FLOATS;
+  uint8_t* blkb = (uint8_t*)ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
   for (int idx = tid; idx < C * DK; idx += 256) {
     const int r = idx / DK, j = idx % DK;
     float kv = 0.f, qv = 0.f;
@@ -298,7 +310,10 @@ __global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q,
     Gs[2 * tid + 1] = x;
   }
   __syncthreads();
-  if (tid < C) blk[WL::G_OFF + tid] = Gs[tid];
+  if (tid < C) {
+    if (WB) reinterpret_cast<float*>(blkb + WLB::G_OFF)[tid] = Gs[tid];
+    else blk[WL::G_OFF + tid] = Gs[tid];
+  }
   {
     // 4 x 4 blocks of K K^T and Q K^T on and below the diagonal
     const int r0 = (tid >> 4) * 4, s0 = (tid & 15) * 4;
@@ -336,7 +351,13 @@ __global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q,
         pv[e] = aq[a][e] * dec;
       }
       *reinterpret_cast<float4*>(As + r * CP + s0) = make_float4(av[0], av[1], av[2], av[3]);
-      *reinterpret_cast<float4*>(blk + WL::P_OFF + r * C + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      if (WB) {
+        __nv_bfloat162* pb = reinterpret_cast<__nv_bfloat162*>(blkb + WLB::P_OFF + (r * C + s0) * 2);
+        pb[0] = __floats2bfloat162_rn(pv[0], pv[1]);
+        pb[1] = __floats2bfloat162_rn(pv[2], pv[3]);
+      } else {
+        *reinterpret_cast<float4*>(blk + WL::P_OFF + r * C + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      }
     }
   }
   __syncthreads();
@@ -365,10 +386,20 @@ __global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q,
       }
       x[r] = acc;
     }
-    float* dst = j < DK ? blk + WL::W_OFF + j : blk + WL::U_OFF + (j - DK);
-    const int stride = j < DK ? DK : DV;
+    if (WB && j < DK) {
+      __nv_bfloat16* wd = reinterpret_cast<__nv_bfloat16*>(blkb + WLB::W_OFF) + j;
 #pragma unroll
-    for (int r = 0; r < C; ++r) dst[r * stride] = x[r];
+      for (int r = 0; r < C; ++r) wd[r * DK] = __float2bfloat16(x[r]);
+    } else if (WB) {
+      float* ud = reinterpret_cast<float*>(blkb + WLB::U_OFF) + (j - DK);
+#pragma unroll
+      for (int r = 0; r < C; ++r) ud[r * DV] = x[r];
+    } else {
+      float* dst = j < DK ? blk + WL::W_OFF + j : blk + WL::U_OFF + (j - DK);
+      const int stride = j < DK ? DK : DV;
+#pragma unroll
+      for (int r = 0; r < C; ++r) dst[r * stride] = x[r];
+    }
   }
 }
 
@@ -546,6 +577,201 @@ __global__ void __launch_bounds__(256) gdn_scan_kernel(const T* __restrict__ q, 
   for (int idx = tid; idx < DVS * DK; idx += 256) Sg[idx] = St[cur][(idx % DK) * DVS + idx / DK];
 }
 
+
+// ------------------------------------------------------------------ tensor-core sequential pass (bf16)
+// The same recurrence as gdn_scan_kernel with the three per-chunk products on the tensor
+// cores (mma.sync m16n8k16, bf16 operands, fp32 accumulation):
+//   U  = U' - W S^T          (64 x 16, K = dk)      A = W,  B = S (bf16 copy)
+//   O  = gamma Q S^T + P U   (64 x 16, K = dk, 64)  A = Q, P; B = S, U
+//   S <- exp(G_last) S + (exp(G_last - G) U)^T K   (16 x dk, K = 64)
+// The fp32 state lives in registers as the accumulator of the last product; each warp
+// owns dk/64 8-column tiles of the 16 state rows of this CTA.
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(su32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(su32(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(su32(p)));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(su32(p)));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float x, float y) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
+}
+
+template <int DK, int DV>
+struct ScanTc {
+  static constexpr int C = GDN_C, DVS = 16, KP = DK + 8, PP = C + 8, UP = DVS + 8;
+  static constexpr int W_B = C * KP * 2, Q_B = W_B, K_B = W_B, P_B = C * PP * 2, UPF_B = C * DVS * 4, G_B = C * 4;
+  static constexpr int STAGE = W_B + Q_B + K_B + P_B + UPF_B + G_B;
+  static constexpr int SB_B = DVS * KP * 2, UB_B = C * UP * 2;
+  static constexpr size_t BYTES = 2 * (size_t)STAGE + SB_B + 2 * UB_B;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* __restrict__ q,
+                                                          const __nv_bfloat16* __restrict__ k,
+                                                          const uint8_t* __restrict__ ws, float* __restrict__ state,
+                                                          __nv_bfloat16* __restrict__ out, int T_len, int H,
+                                                          int n_chunks, float scale) {
+  using L = ScanTc<DK, DV>;
+  using WLB = GdnWsB<DK, DV>;
+  constexpr int C = L::C, DVS = L::DVS, KP = L::KP, PP = L::PP, UP = L::UP;
+  constexpr int NT3 = DK / 64;                               // state column tiles per warp
+  extern __shared__ __align__(16) uint8_t smb[];
+  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + 2 * L::STAGE);  // [DVS][KP] bf16 copy of the state slice
+  __nv_bfloat16* Ub = Sb + DVS * KP;                         // [C][UP] U
+  __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int i0 = blockIdx.x * DVS, h = blockIdx.y, b = blockIdx.z;
+  float* Sg = state + (((long)b * H + h) * DV + i0) * DK;
+
+  float st[NT3][4];
+#pragma unroll
+  for (int j = 0; j < NT3; ++j) {
+    const int col = (w * NT3 + j) * 8 + 2 * tq;
+    st[j][0] = Sg[gq * DK + col];
+    st[j][1] = Sg[gq * DK + col + 1];
+    st[j][2] = Sg[(gq + 8) * DK + col];
+    st[j][3] = Sg[(gq + 8) * DK + col + 1];
+    st_bf2(Sb + gq * KP + col, st[j][0], st[j][1]);
+    st_bf2(Sb + (gq + 8) * KP + col, st[j][2], st[j][3]);
+  }
+
+  auto issue = [&](int c, int bi) {
+    uint8_t* base = smb + bi * L::STAGE;
+    const uint8_t* blk = ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
+    const int c0 = c * C, n = min(C, T_len - c0);
+    constexpr int RP = DK * 2 / 16;                          // 16-byte pieces per row
+    for (int idx = tid; idx < C * RP; idx += 256) {
+      const int r = idx / RP, p = idx % RP;
+      cp_async16(base + r * KP * 2 + 16 * p, blk + WLB::W_OFF + r * DK * 2 + 16 * p, true);
+      const bool ok = r < n;
+      const long row = (((long)b * T_len + c0 + (ok ? r : 0)) * H + h) * DK;
+      cp_async16(base + L::W_B + r * KP * 2 + 16 * p, (const uint8_t*)(q + row) + 16 * p, ok);
+      cp_async16(base + L::W_B + L::Q_B + r * KP * 2 + 16 * p, (const uint8_t*)(k + row) + 16 * p, ok);
+    }
+    for (int idx = tid; idx < C * (C * 2 / 16); idx += 256) {
+      const int r = idx / (C * 2 / 16), p = idx % (C * 2 / 16);
+      cp_async16(base + L::W_B + L::Q_B + L::K_B + r * PP * 2 + 16 * p, blk + WLB::P_OFF + r * C * 2 + 16 * p, true);
+    }
+    for (int idx = tid; idx < C * DVS / 4; idx += 256) {
+      const int r = idx / (DVS / 4), p = idx % (DVS / 4);
+      cp_async16(base + L::W_B + L::Q_B + L::K_B + L::P_B + r * DVS * 4 + 16 * p,
+                 blk + WLB::U_OFF + (r * DV + i0) * 4 + 16 * p, true);
+    }
+    if (tid < C / 4)
+      cp_async16(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B + 16 * tid, blk + WLB::G_OFF + 16 * tid, true);
+    cp_async_commit();
+  };
+
+  issue(0, 0);
+  const int mt = w >> 1, nt = w & 1;                         // phases 1-2: 4 x 2 output tiles
+  const int r0 = mt * 16 + gq, r1 = r0 + 8, ic = nt * 8 + 2 * tq;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int bi = c & 1;
+    if (c + 1 < n_chunks) {
+      issue(c + 1, bi ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t* base = smb + bi * L::STAGE;
+    const __nv_bfloat16* Wb = (const __nv_bfloat16*)base;
+    const __nv_bfloat16* Qb = (const __nv_bfloat16*)(base + L::W_B);
+    const __nv_bfloat16* Kb = (const __nv_bfloat16*)(base + L::W_B + L::Q_B);
+    const __nv_bfloat16* Pb = (const __nv_bfloat16*)(base + L::W_B + L::Q_B + L::K_B);
+    const float* Upf = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B);
+    const float* Gs = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
+    const int c0 = c * C, n = min(C, T_len - c0);
+    const float Glast = Gs[C - 1];
+    // phase 1 + 2a: W S^T and Q S^T share the B operand
+    float cu[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < DK / 16; ++ks) {
+      uint32_t aw[4], aq[4], bs[2];
+      ldsm_x4(aw, Wb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
+      ldsm_x4(aq, Qb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
+      ldsm_x2(bs, Sb + (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8);
+      mma16816(cu, aw, bs);
+      mma16816(cq, aq, bs);
+    }
+    {
+      const float u00 = Upf[r0 * DVS + ic] - cu[0], u01 = Upf[r0 * DVS + ic + 1] - cu[1];
+      const float u10 = Upf[r1 * DVS + ic] - cu[2], u11 = Upf[r1 * DVS + ic + 1] - cu[3];
+      const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
+      st_bf2(Ub + r0 * UP + ic, u00, u01);
+      st_bf2(Ub + r1 * UP + ic, u10, u11);
+      st_bf2(Ueb + r0 * UP + ic, u00 * e0, u01 * e0);
+      st_bf2(Ueb + r1 * UP + ic, u10 * e1, u11 * e1);
+    }
+    __syncthreads();
+    // phase 2b: P U, then the outputs
+    float cp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      uint32_t ap[4], bu[2];
+      ldsm_x4(ap, Pb + (mt * 16 + (lane & 15)) * PP + ks * 16 + (lane >> 4) * 8);
+      ldsm_x2_t(bu, Ub + (ks * 16 + (lane & 15)) * UP + nt * 8);
+      mma16816(cp, ap, bu);
+    }
+    {
+      const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]);
+      if (r0 < n)
+        st_bf2(out + (((long)b * T_len + c0 + r0) * H + h) * DV + i0 + ic, scale * fmaf(g0, cq[0], cp[0]),
+               scale * fmaf(g0, cq[1], cp[1]));
+      if (r1 < n)
+        st_bf2(out + (((long)b * T_len + c0 + r1) * H + h) * DV + i0 + ic, scale * fmaf(g1, cq[2], cp[2]),
+               scale * fmaf(g1, cq[3], cp[3]));
+    }
+    // phase 3: S <- exp(G_last) S + Ue^T K
+    const float gl = expf(Glast);
+#pragma unroll
+    for (int j = 0; j < NT3; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[j][e] *= gl;
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      uint32_t au[4];
+      ldsm_x4_t(au, Ueb + (ks * 16 + (lane >> 4) * 8 + (lane & 7)) * UP + ((lane >> 3) & 1) * 8);
+#pragma unroll
+      for (int j = 0; j < NT3; ++j) {
+        uint32_t bk[2];
+        ldsm_x2_t(bk, Kb + (ks * 16 + (lane & 15)) * KP + (w * NT3 + j) * 8);
+        mma16816(st[j], au, bk);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT3; ++j) {
+      const int col = (w * NT3 + j) * 8 + 2 * tq;
+      st_bf2(Sb + gq * KP + col, st[j][0], st[j][1]);
+      st_bf2(Sb + (gq + 8) * KP + col, st[j][2], st[j][3]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < NT3; ++j) {
+    const int col = (w * NT3 + j) * 8 + 2 * tq;
+    Sg[gq * DK + col] = st[j][0];
+    Sg[gq * DK + col + 1] = st[j][1];
+    Sg[(gq + 8) * DK + col] = st[j][2];
+    Sg[(gq + 8) * DK + col + 1] = st[j][3];
+  }
+}
+
 template <typename T, int DK, int DV>
 static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                    float* state, void* out, int B, int T_len, int H, float scale, void* workspace,
@@ -553,13 +779,17 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
   constexpr int DVS = 16;
   const int n_chunks = (T_len + GDN_C - 1) / GDN_C;
   const size_t smem1 = (size_t)(2 * DK * (GDN_C + 4) + GDN_C * (GDN_C + 4) + 2 * GDN_C) * sizeof(float);
-  auto k1 = gdn_intra_kernel<T, DK, DV>;
+  constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;   // bf16: tensor-core sequential pass
+  auto k1 = gdn_intra_kernel<T, DK, DV, TC>;
   auto k2 = gdn_scan_kernel<T, DK, DV, DVS>;
+  auto k2t = gdn_scan_tc_kernel<DK, DV>;
   using L = ScanSmem<T, DK, DV, DVS>;
+  using LT = ScanTc<DK, DV>;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k2t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LT::BYTES);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -567,8 +797,13 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
                                                H, n_chunks);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,
-                                                  T_len, H, n_chunks, scale);
+  if (TC)
+    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                          (const uint8_t*)workspace, state, (__nv_bfloat16*)out, T_len,
+                                                          H, n_chunks, scale);
+  else
+    k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,
+                                                    T_len, H, n_chunks, scale);
   return cudaGetLastError();
 }
 

@@ -63,9 +63,11 @@ cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, i
                         int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
                         cudaStream_t s);
 
+// w_rt: optional [8, 2d] transposed copy of w_r (coalesced routing-map reads).
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
                 const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,
-                int d, float eps, int iters, int dtype, cudaStream_t s);
+                int d, float eps, int iters, int dtype, cudaStream_t s, const float* w_rt = nullptr);
+cudaError_t transpose_wr(const float* w, float* wt, int two_d, cudaStream_t s);
 cudaError_t sinkhorn(const float* logits, float* out, int N, int n, int iters, cudaStream_t s);
 
 int read_and_clear_device_error();

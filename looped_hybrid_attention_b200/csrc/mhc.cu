@@ -4,9 +4,10 @@
 // Sinkhorn) and reads the layer input -- the streams cross HBM once per boundary.
 //
 // A warp owns 4 consecutive tokens.  Lane L owns elements [8L + 256c, 8L + 256c + 8)
-// of each stream (16-byte accesses), so the 2x[d] stream pairs and the [2d, 8] routing
-// map are read fully coalesced, and each routing-map row loaded serves all 4 tokens
-// (the map is 256 KiB at d = 4096 and stays in L2).
+// of each stream (16-byte accesses).  The routing map is read through its transposed
+// copy [8, 2d] (w_rt, kept by the model) so that, per output, the warp reads one
+// contiguous 1 KiB run; each value loaded serves all 4 tokens.  The per-op entry
+// point, which has only the [2d, 8] map, reads it directly.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,7 +23,7 @@ __device__ __forceinline__ void sinkhorn2(float m[4], int iters) {
   }
 }
 
-template <typename T, int TPW>
+template <typename T, int TPW, bool WT>
 __global__ void __launch_bounds__(128) mhc_kernel(int mode, const T* __restrict__ X_in, const T* __restrict__ F,
                                                   const float* __restrict__ coeffs_in,
                                                   const float* __restrict__ w_r, const float* __restrict__ b_r,
@@ -100,22 +101,41 @@ __global__ void __launch_bounds__(128) mhc_kernel(int mode, const T* __restrict_
       for (int i = 0; i < 8; ++i) ss[t] += y0[t][i] * y0[t][i] + y1[t][i] * y1[t][i];
     }
     if (mode == MHC_MERGE) continue;
+    if (WT) {
+      // transposed map: output o reads w_r[o][j .. j+8) and w_r[o][d+j .. d+j+8), coalesced
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4* w0 = reinterpret_cast<const float4*>(w_r + (long)(j + i) * 8);
-      const float4* w1 = reinterpret_cast<const float4*>(w_r + (long)(d + j + i) * 8);
-      const float4 a0 = __ldg(w0), a1 = __ldg(w0 + 1), b0 = __ldg(w1), b1 = __ldg(w1 + 1);
+      for (int o = 0; o < 8; ++o) {
+        const float4* wa = reinterpret_cast<const float4*>(w_r + (long)o * 2 * d + j);
+        const float4* wb = reinterpret_cast<const float4*>(w_r + (long)o * 2 * d + d + j);
+        const float4 a0 = __ldg(wa), a1 = __ldg(wa + 1), b0 = __ldg(wb), b1 = __ldg(wb + 1);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int t = 0; t < TPW; ++t) {
-        const float u = y0[t][i], v = y1[t][i];
-        l[t][0] += u * a0.x + v * b0.x;
-        l[t][1] += u * a0.y + v * b0.y;
-        l[t][2] += u * a0.z + v * b0.z;
-        l[t][3] += u * a0.w + v * b0.w;
-        l[t][4] += u * a1.x + v * b1.x;
-        l[t][5] += u * a1.y + v * b1.y;
-        l[t][6] += u * a1.z + v * b1.z;
-        l[t][7] += u * a1.w + v * b1.w;
+        for (int t = 0; t < TPW; ++t) {
+          float acc = l[t][o];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc += y0[t][i] * av[i] + y1[t][i] * bv[i];
+          l[t][o] = acc;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4* w0 = reinterpret_cast<const float4*>(w_r + (long)(j + i) * 8);
+        const float4* w1 = reinterpret_cast<const float4*>(w_r + (long)(d + j + i) * 8);
+        const float4 a0 = __ldg(w0), a1 = __ldg(w0 + 1), b0 = __ldg(w1), b1 = __ldg(w1 + 1);
+#pragma unroll
+        for (int t = 0; t < TPW; ++t) {
+          const float u = y0[t][i], v = y1[t][i];
+          l[t][0] += u * a0.x + v * b0.x;
+          l[t][1] += u * a0.y + v * b0.y;
+          l[t][2] += u * a0.z + v * b0.z;
+          l[t][3] += u * a0.w + v * b0.w;
+          l[t][4] += u * a1.x + v * b1.x;
+          l[t][5] += u * a1.y + v * b1.y;
+          l[t][6] += u * a1.z + v * b1.z;
+          l[t][7] += u * a1.w + v * b1.w;
+        }
       }
     }
   }
@@ -278,9 +298,23 @@ __global__ void __launch_bounds__(512) mhc_token_kernel(int mode, const T* __res
   }
 }
 
+// w_r [8, 2d] from the [2d, 8] routing map (run once per looped layer by the model).
+__global__ void transpose_wr_kernel(const float* __restrict__ w, float* __restrict__ wt, int rows) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)rows * 8) return;
+  const long r = i / 8, o = i % 8;
+  wt[o * rows + r] = w[i];
+}
+
+cudaError_t transpose_wr(const float* w, float* wt, int two_d, cudaStream_t s) {
+  const long n = (long)two_d * 8;
+  transpose_wr_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w, wt, two_d);
+  return cudaGetLastError();
+}
+
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,
                 const float* b_r, void* X_out, void* x_in, void* h_out, float* coeffs_out, int N,
-                int d, float eps, int iters, int dtype, cudaStream_t s) {
+                int d, float eps, int iters, int dtype, cudaStream_t s, const float* w_rt) {
   if (N == 0) return cudaSuccess;
   if (N < 1024) {           // few tokens: spread each token over a CTA
     const int threads = d >= 4096 ? 512 : (d >= 2048 ? 256 : 128);
@@ -296,14 +330,17 @@ cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_i
   }
   constexpr int TPW = 4, warps = 4;
   dim3 grid((unsigned)(((long)N + TPW * warps - 1) / (TPW * warps)));
-  if (dtype == BF16)
-    mhc_kernel<__nv_bfloat16, TPW><<<grid, warps * 32, 0, s>>>(
-        mode, (const __nv_bfloat16*)X_in, (const __nv_bfloat16*)F, coeffs_in, w_r, b_r,
-        (__nv_bfloat16*)X_out, (__nv_bfloat16*)x_in, (__nv_bfloat16*)h_out, coeffs_out, N, d, eps, iters);
-  else
-    mhc_kernel<float, TPW><<<grid, warps * 32, 0, s>>>(mode, (const float*)X_in, (const float*)F, coeffs_in,
-                                                       w_r, b_r, (float*)X_out, (float*)x_in, (float*)h_out,
-                                                       coeffs_out, N, d, eps, iters);
+  const bool wt = w_rt != nullptr;
+  const float* wmap = wt ? w_rt : w_r;
+#define MHC_LAUNCH(TT, W)                                                                                            \
+  mhc_kernel<TT, TPW, W><<<grid, warps * 32, 0, s>>>(mode, (const TT*)X_in, (const TT*)F, coeffs_in, wmap, b_r,      \
+                                                     (TT*)X_out, (TT*)x_in, (TT*)h_out, coeffs_out, N, d, eps, iters)
+  if (dtype == BF16) {
+    if (wt) MHC_LAUNCH(__nv_bfloat16, true); else MHC_LAUNCH(__nv_bfloat16, false);
+  } else {
+    if (wt) MHC_LAUNCH(float, true); else MHC_LAUNCH(float, false);
+  }
+#undef MHC_LAUNCH
   return cudaGetLastError();
 }
 

@@ -246,6 +246,8 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
   return LOOP_OK;
 }
 
+static const float* wr_t(loop_model* m, int layer);
+
 // All executions over M = B*T new tokens whose hidden states are in m->h.
 static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStream_t s) {
   const loop_config& cf = m->cfg;
@@ -264,7 +266,8 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
     if (r.exec == m->first_loop)
       CK(prof(m, s, P_MHC, 1, 0, tok * (es * 4.0 * cf.d + 32.0),
               [&] { return mhc(MHC_OPEN, m->h.p, nullptr, nullptr, w.mhc_w_r, w.mhc_b_r, m->X.p, m->x_in.p, nullptr,
-                               (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
+                               (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s,
+                               wr_t(m, r.layer)); }),
          "mHC open");
     loop_status st = run_layer(m, c, r, m->x_in.p, nullptr, B, T, pos0, s);
     if (st != LOOP_OK) return st;
@@ -278,11 +281,30 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
       // read X (2d) + F (d), write X' (2d) + x_in (d), coefficients in/out
       CK(prof(m, s, P_MHC, 1, 0, tok * (es * 6.0 * cf.d + 64.0),
               [&] { return mhc(MHC_MIX, m->X.p, m->F.p, (float*)m->coeffs.p, wn.mhc_w_r, wn.mhc_b_r, m->X.p, m->x_in.p,
-                               nullptr, (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
+                               nullptr, (float*)m->coeffs.p, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s,
+                               wr_t(m, m->sched[i + 1].layer)); }),
          "mHC mix + route");
     }
   }
   return LOOP_OK;
+}
+
+// One-time preparation on the first forward (on the caller's stream): transposed copies
+// of the looped layers' routing maps.
+static loop_status prepare(loop_model* m, cudaStream_t s) {
+  if (m->wrt_ready) return LOOP_OK;
+  const loop_config& c = m->cfg;
+  const size_t per = (size_t)2 * c.d * 8;
+  CK(m->wrt.ensure(std::max<size_t>(256, (size_t)c.n_layers * per * sizeof(float))), "routing-map copy allocation");
+  for (int l = 0; l < c.n_layers; ++l)
+    if (m->layers[l].mhc_w_r)
+      CK(transpose_wr(m->layers[l].mhc_w_r, (float*)m->wrt.p + l * per, 2 * c.d, s), "routing-map transpose");
+  m->wrt_ready = true;
+  return LOOP_OK;
+}
+
+static const float* wr_t(loop_model* m, int layer) {
+  return (const float*)m->wrt.p + (size_t)layer * 2 * m->cfg.d * 8;
 }
 
 loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const void* h_in, void* h_out,
@@ -290,6 +312,8 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
   const loop_config& cf = m->cfg;
   const long M = (long)B * T;
   loop_status st = ensure_workspace(m, M, B, T, c->max_tokens);
+  if (st != LOOP_OK) return st;
+  st = prepare(m, s);
   if (st != LOOP_OK) return st;
   const double es = (double)m->esize;
   if (ids)
@@ -324,6 +348,8 @@ loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* 
   const loop_config& cf = m->cfg;
   const int B = c->batch;
   loop_status st = ensure_workspace(m, B, B, 1, c->max_tokens);
+  if (st != LOOP_OK) return st;
+  st = prepare(m, s);
   if (st != LOOP_OK) return st;
   // logits go to the caller's buffer if given, else to a workspace buffer
   float* lg = logits;

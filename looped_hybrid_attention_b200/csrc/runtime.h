@@ -55,6 +55,8 @@ struct loop_model {
   DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, gdn_ws, gemm_ws, last;
   int in_gdn = 0, in_fa = 0;
   Profiler prof;
+  DevBuf wrt;                    // [n_layers][8][2d] transposed routing maps (looped layers)
+  bool wrt_ready = false;
 };
 
 struct loop_cache {

@@ -123,3 +123,19 @@ def test_group_bf16_vs_oracle(cuda):
     m.forward_hidden(c, h.cuda(), out)
     torch.cuda.synchronize()
     assert rel_l2(to64(out), ref) < TOL["bf16_e2e"]
+
+
+def test_tiny_stack_long_sequence_fp32(cuda):
+    """1100 tokens: the prefill-sized mHC path (4 tokens per warp, transposed routing maps) and many GDN chunks."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.TINY
+    w = synth.make_weights(s, seed=5)
+    T = 1100
+    h = synth.normal((1, T, s.d), 1.0, 5, "hidden")
+    ref, _ = omodel.forward_hidden(s, omodel.Weights(w), h)
+    m = L.Model(s, dev_weights(w))
+    c = m.cache(1, T)
+    out = torch.empty((1, T, s.d), device=cuda)
+    m.forward_hidden(c, h.cuda(), out)
+    torch.cuda.synchronize()
+    assert rel_l2(to64(out), ref) < TOL["fp32"]
