@@ -416,6 +416,234 @@ static cudaError_t launch_decode(const void* q, int ld_q, const void* k, const v
   return cudaGetLastError();
 }
 
+
+// ------------------------------------------------------------------ single-token decode on tensor cores
+// The same flash-decode with the products on mma.sync (m16n8k16, bf16 -> fp32): the
+// q heads of one KV group are the rows of a 16-row A tile (rows >= Hq/Hkv are zero).
+// Per 64-key tile: warp w computes S for keys [16w, 16w+16) (Q fragments stay in
+// registers), the tile's row max and sum are combined through shared memory, then warp
+// w accumulates O for head dims [w*DH/4, (w+1)*DH/4) with P from shared memory.
+constexpr int DTC_KT = 64, DTC_STAGES = 3;
+
+template <int DH>
+struct DecTc {
+  static constexpr int ROW = DH * 2 + 16;                   // padded K / V row (bytes)
+  static constexpr int STAGE = 2 * DTC_KT * ROW;
+  static constexpr int QROW = DH * 2 + 16;
+  static constexpr int PROW = DTC_KT * 2 + 16;
+  static constexpr size_t BYTES = (size_t)DTC_STAGES * STAGE + 16 * QROW + 16 * PROW + 2 * 4 * 16 * 4;
+};
+
+__device__ __forceinline__ uint32_t sa32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void lds_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(sa32(p)));
+}
+__device__ __forceinline__ void lds_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(sa32(p)));
+}
+__device__ __forceinline__ void hmma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int DH>
+__global__ void __launch_bounds__(128) attn_decode_tc_kernel(const __nv_bfloat16* __restrict__ q, int ld_q,
+                                                             const __nv_bfloat16* __restrict__ kc,
+                                                             const __nv_bfloat16* __restrict__ vc, int kv_cap,
+                                                             const __nv_bfloat16* __restrict__ gate, int ld_gate,
+                                                             __nv_bfloat16* __restrict__ out, float* __restrict__ ws,
+                                                             int Tkv, int q_off, int Hq, int Hkv, int causal,
+                                                             int n_split, int split_len, float scale_log2) {
+  using L = DecTc<DH>;
+  constexpr int CH = DH / 8;                                 // 16-byte chunks per K/V row
+  constexpr int WD = DH / 4;                                 // head dims per warp in P.V
+  constexpr int NTO = WD / 8;                                // 8-wide output tiles per warp
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint8_t* sQ = sm + DTC_STAGES * L::STAGE;                  // [16][QROW] bf16
+  uint8_t* sP = sQ + 16 * L::QROW;                           // [16][PROW] bf16
+  float* sMax = (float*)(sP + 16 * L::PROW);                 // [4 warps][16 rows]
+  float* sSum = sMax + 4 * 16;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int rep = Hq / Hkv;
+  for (int i = tid; i < 16 * CH; i += 128) {
+    const int r = i / CH, c = i % CH;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < rep) val = *reinterpret_cast<const uint4*>(q + (long)b * ld_q + (long)(kvh * rep + r) * DH + c * 8);
+    *reinterpret_cast<uint4*>(sQ + r * L::QROW + c * 16) = val;
+  }
+  int k_end = Tkv;
+  if (causal) k_end = min(k_end, q_off + 1);
+  const int k_begin = split * split_len;
+  k_end = min(k_end, k_begin + split_len);
+  const int n_tiles = k_end > k_begin ? (k_end - k_begin + DTC_KT - 1) / DTC_KT : 0;
+  const __nv_bfloat16* Kb = kc + ((long)b * Hkv + kvh) * kv_cap * DH;
+  const __nv_bfloat16* Vb = vc + ((long)b * Hkv + kvh) * kv_cap * DH;
+  auto issue = [&](int t) {
+    uint8_t* st = sm + (t % DTC_STAGES) * L::STAGE;
+    const int key0 = k_begin + t * DTC_KT;
+    for (int i = tid; i < DTC_KT * CH; i += 128) {
+      const int r = i / CH, c = i % CH;
+      const int key = key0 + r;
+      const bool ok = key < k_end;
+      const long off = (long)(ok ? key : k_begin) * DH + c * 8;
+      cpa16(st + r * L::ROW + c * 16, Kb + off, ok);
+      cpa16(st + DTC_KT * L::ROW + r * L::ROW + c * 16, Vb + off, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+#pragma unroll
+  for (int t = 0; t < DTC_STAGES - 1; ++t) {
+    if (t < n_tiles) issue(t);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  __syncthreads();
+  uint32_t qa[DH / 16][4];                                   // Q fragments for every 16-dim step
+#pragma unroll
+  for (int ks = 0; ks < DH / 16; ++ks) lds_x4(qa[ks], sQ + (lane & 15) * L::QROW + (ks * 16 + (lane >> 4) * 8) * 2);
+  float o[NTO][4];
+#pragma unroll
+  for (int j = 0; j < NTO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;                      // row gq (rows gq+8 are padding)
+  for (int t = 0; t < n_tiles; ++t) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(DTC_STAGES - 2) : "memory");
+    __syncthreads();
+    const uint8_t* st = sm + (t % DTC_STAGES) * L::STAGE;
+    const uint8_t* vt = st + DTC_KT * L::ROW;
+    // S for keys [16w, 16w + 16): two 8-key tiles
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < DH / 16; ks += 2) {
+      uint32_t kb0[4], kb1[4];
+      // keys 16w + (lane & 7) (+8 for the second tile), dims ks*16 .. ks*16 + 32
+      lds_x4(kb0, st + (w * 16 + (lane & 7)) * L::ROW + (ks * 16 + (lane >> 3) * 8) * 2);
+      lds_x4(kb1, st + (w * 16 + 8 + (lane & 7)) * L::ROW + (ks * 16 + (lane >> 3) * 8) * 2);
+      hmma(sc[0], qa[ks], kb0[0], kb0[1]);
+      hmma(sc[1], qa[ks], kb1[0], kb1[1]);
+      hmma(sc[0], qa[ks + 1], kb0[2], kb0[3]);
+      hmma(sc[1], qa[ks + 1], kb1[2], kb1[3]);
+    }
+    const int kbase = k_begin + t * DTC_KT + w * 16 + 2 * tq;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = kbase + j * 8 + e;
+        sc[j][e] = key < k_end ? sc[j][e] * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[j][e]);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (tq == 0) sMax[w * 16 + gq] = mx;
+    __syncthreads();
+    const float tmax = fmaxf(fmaxf(sMax[gq], sMax[16 + gq]), fmaxf(sMax[32 + gq], sMax[48 + gq]));
+    const float m_new = fmaxf(m_run, tmax);
+    const float corr = exp2f(m_run - m_new);
+    float ps = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float p0 = exp2f(sc[j][0] - m_new), p1 = exp2f(sc[j][1] - m_new);
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+      const float2 pf = __bfloat1622float2(pb);
+      ps += pf.x + pf.y;
+      *reinterpret_cast<__nv_bfloat162*>(sP + gq * L::PROW + (w * 16 + j * 8 + 2 * tq) * 2) = pb;
+      *reinterpret_cast<__nv_bfloat162*>(sP + (gq + 8) * L::PROW + (w * 16 + j * 8 + 2 * tq) * 2) =
+          __floats2bfloat162_rn(0.f, 0.f);
+    }
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+    if (tq == 0) sSum[w * 16 + gq] = ps;
+    __syncthreads();
+    l_run = l_run * corr + (sSum[gq] + sSum[16 + gq] + sSum[32 + gq] + sSum[48 + gq]);
+    m_run = m_new;
+#pragma unroll
+    for (int j = 0; j < NTO; ++j) {
+      o[j][0] *= corr;
+      o[j][1] *= corr;
+    }
+    // O[:, w*WD .. +WD) += P V
+#pragma unroll
+    for (int ks = 0; ks < DTC_KT / 16; ++ks) {
+      uint32_t pa[4];
+      lds_x4(pa, sP + (lane & 15) * L::PROW + (ks * 16 + (lane >> 4) * 8) * 2);
+#pragma unroll
+      for (int j = 0; j < NTO; j += 2) {
+        uint32_t vb[4];
+        // rows ks*16 + (lane & 15) of V, dims w*WD + j*8 (+8 for lanes 16..31)
+        lds_x4_t(vb, vt + (ks * 16 + (lane & 15)) * L::ROW + (w * WD + j * 8 + (lane >> 4) * 8) * 2);
+        hmma(o[j], pa, vb[0], vb[1]);
+        hmma(o[j + 1], pa, vb[2], vb[3]);
+      }
+    }
+    __syncthreads();
+    if (t + DTC_STAGES - 1 < n_tiles) issue(t + DTC_STAGES - 1);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  if (gq >= rep) return;
+  const int h = kvh * rep + gq;
+  if (n_split == 1) {
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int j = 0; j < NTO; ++j) {
+      const int dcol = w * WD + j * 8 + 2 * tq;
+      float v0 = o[j][0] * inv, v1 = o[j][1] * inv;
+      if (gate) {
+        const __nv_bfloat16* gp = gate + (long)b * ld_gate + (long)h * DH + dcol;
+        v0 *= sigmoidf_acc(__bfloat162float(gp[0]));
+        v1 *= sigmoidf_acc(__bfloat162float(gp[1]));
+      }
+      *reinterpret_cast<__nv_bfloat162*>(out + ((long)b * Hq + h) * DH + dcol) = __floats2bfloat162_rn(v0, v1);
+    }
+  } else {
+    // partials in the split-K layout: (max in natural-log units, sum, o[DH])
+    float* wp = ws + (((long)b * Hq + h) * n_split + split) * (DH + 2);
+    if (w == 0 && tq == 0) {
+      wp[0] = m_run / 1.4426950408889634f;
+      wp[1] = l_run;
+    }
+#pragma unroll
+    for (int j = 0; j < NTO; ++j) {
+      const int dcol = w * WD + j * 8 + 2 * tq;
+      wp[2 + dcol] = o[j][0];
+      wp[3 + dcol] = o[j][1];
+    }
+  }
+}
+
+template <int DH>
+static cudaError_t launch_decode_tc(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                                   const void* gate, int ld_gate, void* out, int B, int Tkv, int q_off, int Hq, int Hkv,
+                                   int causal, void* workspace, cudaStream_t s) {
+  using L = DecTc<DH>;
+  const int n_split = workspace ? attn_splits(B, 1, Tkv, Hkv) : 1;
+  const int split_len = (((Tkv + n_split - 1) / n_split) + DTC_KT - 1) / DTC_KT * DTC_KT;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(n_split, Hkv, B);
+  attn_decode_tc_kernel<DH><<<grid, 128, L::BYTES, s>>>(
+      (const __nv_bfloat16*)q, ld_q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, kv_cap,
+      (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, (float*)workspace, Tkv, q_off, Hq, Hkv, causal,
+      n_split, split_len, 1.4426950408889634f / sqrtf((float)DH));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || n_split == 1) return e;
+  const long rows = (long)B * Hq;
+  attn_combine_kernel<__nv_bfloat16, DH><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+      (const float*)workspace, (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, rows, Hq, n_split);
+  return cudaGetLastError();
+}
+
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
   const int Hkv = 1;   // upper bound: splits computed with Hkv = 1 are never fewer
   const int s = attn_splits(B, Tq, Tkv, Hkv);
@@ -463,6 +691,12 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
     if (e != cudaErrorNotSupported) return e;
   }
   // single-token decode (bf16, <= 4 q heads per KV head): the tiled flash-decode kernel
+  if (Tq == 1 && dtype == BF16 && Hq / Hkv <= 16 && (dh == 256 || dh == 128) && ((uintptr_t)k % 16 == 0) &&
+      ((uintptr_t)v % 16 == 0) && ((uintptr_t)q % 16 == 0) && ld_q % 8 == 0) {
+    if (dh == 256)
+      return launch_decode_tc<256>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
+    return launch_decode_tc<128>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
+  }
   if (Tq == 1 && dtype == BF16 && Hq / Hkv <= 4 && (dh == 256 || dh == 128 || dh == 64) &&
       ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0)) {
     if (dh == 256)
