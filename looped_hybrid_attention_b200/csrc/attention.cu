@@ -16,12 +16,34 @@
 namespace lk {
 
 // ------------------------------------------------------------------ QK-norm + rotary + KV write
+// cos/sin of pos * base^(-2j/rot) for positions pos0 .. pos0+T-1 and pairs j < rot/2,
+// evaluated in fp64 (angles reach 1e5 rad at long context) and stored as fp32 pairs.
+__global__ void rope_table_kernel(float2* __restrict__ tab, int T_len, int pos0, int rot, float base) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int half = rot / 2;
+  if (i >= (long)T_len * half) return;
+  const int t = (int)(i / half), j = (int)(i % half);
+  const double theta = pow((double)base, -2.0 * (double)j / (double)rot);
+  double ang = (double)(pos0 + t) * theta;
+  ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  tab[i] = make_float2((float)cs, (float)sn);
+}
+
+cudaError_t rope_table(float2* tab, int T, int pos0, int rot, float base, cudaStream_t s) {
+  const long n = (long)T * (rot / 2);
+  if (n == 0) return cudaSuccess;
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, T, pos0, rot, base);
+  return cudaGetLastError();
+}
+
 template <typename T, int DH>
 __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, int ld_p, const T* __restrict__ q_norm,
                                                       const T* __restrict__ k_norm, T* __restrict__ q_out,
                                                       T* __restrict__ k_cache, T* __restrict__ v_cache, int kv_cap,
                                                       int T_len, int pos0, int Hq, int Hkv, int rot, float base,
-                                                      float eps) {
+                                                      float eps, const float2* __restrict__ tab) {
   constexpr int PER = DH / 32;         // contiguous elements per lane (even: rotary pairs stay local)
   const int lane = threadIdx.x & 31;
   const int heads = Hq + Hkv;
@@ -51,12 +73,20 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
     const int e = lane * PER + u;
     if (e < rot) {
       const int j = e >> 1;
-      const double theta = pow((double)base, -2.0 * (double)j / (double)rot);
-      double ang = (double)pos * theta;
-      ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      const float c = (float)cs, s = (float)sn;
+      float c, s;
+      if (tab) {
+        const float2 cs2 = tab[(long)t * (rot / 2) + j];
+        c = cs2.x;
+        s = cs2.y;
+      } else {
+        const double theta = pow((double)base, -2.0 * (double)j / (double)rot);
+        double ang = (double)pos * theta;
+        ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        c = (float)cs;
+        s = (float)sn;
+      }
       const float a0 = x[u], a1 = x[u + 1];
       x[u] = a0 * c - a1 * s;
       x[u + 1] = a0 * s + a1 * c;
@@ -80,7 +110,7 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
 cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
                     void* k_cache, void* v_cache, int kv_cap, int B, int T, int pos0, int Hq,
                     int Hkv, int dh, int rotary_dims, float rope_base, float eps, int dtype,
-                    cudaStream_t s) {
+                    cudaStream_t s, const float2* rope_tab) {
   if (T == 0 || B == 0) return cudaSuccess;
   const int warps = 8;
   dim3 grid((unsigned)(((long)T * (Hq + Hkv) + warps - 1) / warps), B);
@@ -88,7 +118,7 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
   fa_prep_kernel<TT, DHV><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,               \
                                                       (const TT*)k_norm, (TT*)q_out, (TT*)k_cache,         \
                                                       (TT*)v_cache, kv_cap, T, pos0, Hq, Hkv, rotary_dims, \
-                                                      rope_base, eps)
+                                                      rope_base, eps, rope_tab)
   if (dtype == BF16) {
     if (dh == 256) FA_PREP(__nv_bfloat16, 256); else if (dh == 128) FA_PREP(__nv_bfloat16, 128);
     else if (dh == 64) FA_PREP(__nv_bfloat16, 64); else return cudaErrorNotSupported;

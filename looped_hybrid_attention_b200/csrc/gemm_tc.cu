@@ -277,14 +277,15 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int spli
   }
 }
 
-// K-slices for a GEMM with few output tiles (small M): aim for two units per SM, keep
-// at least 4 K-blocks per slice, and fit the partials in `ws_bytes`.
+// K-slices for a GEMM with few output tiles (small M): aim for one unit per SM (more
+// slices only add partial-sum traffic), keep at least 4 K-blocks per slice, and fit
+// the partials in `ws_bytes`.
 static int choose_splits(int M, int N, int K, int epi, size_t ws_bytes) {
   constexpr int BN = 256;
   const int out_cols = epi == EPI_SWIGLU ? BN / 2 : BN;
   const long tiles = (long)((M + BM - 1) / BM) * ((N + out_cols - 1) / out_cols);
   const int kb = (K + BK - 1) / BK;
-  int sp = (int)((2L * num_sms() + tiles - 1) / tiles);
+  int sp = (int)((num_sms() + tiles - 1) / tiles);
   sp = min(sp, kb / 4);
   sp = min(sp, 16);
   const long nc = epi == EPI_SWIGLU ? 2L * N : N;

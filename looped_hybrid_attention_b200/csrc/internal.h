@@ -45,10 +45,12 @@ cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g
                      cudaStream_t s);
 bool gdn_supported(int dk, int dv);
 
+// rope_tab: optional [T, rotary_dims/2] (cos, sin) table from rope_table (else fp64 in-kernel).
 cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
                     void* k_cache, void* v_cache, int kv_cap, int B, int T, int pos0, int Hq,
                     int Hkv, int dh, int rotary_dims, float rope_base, float eps, int dtype,
-                    cudaStream_t s);
+                    cudaStream_t s, const float2* rope_tab = nullptr);
+cudaError_t rope_table(float2* tab, int T, int pos0, int rot, float base, cudaStream_t s);
 cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
                      const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,

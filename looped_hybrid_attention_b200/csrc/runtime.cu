@@ -126,6 +126,7 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->act, M * c.ffn * es},
       {&m->F, M * d * es},
       {&m->coeffs, M * 8 * sizeof(float)},
+      {&m->rope, (size_t)Tq * (c.rotary_dims / 2) * sizeof(float2)},
       {&m->attn_ws, gqa_workspace_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_head_dim)},
       {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
       // split-K partials for projections with few tokens (the widest: the FFN gate/up pair)
@@ -212,7 +213,8 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
     char* vbase = kbase + c->kv_slab_elems * m->esize;
     CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * (Hq + 2 * Hkv) * dh),
             [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, m->gq.p, kbase, vbase, c->max_tokens, B, T,
-                                     pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt, s); }),
+                                     pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt, s,
+                                     (const float2*)m->rope.p); }),
        "QK-norm / rotary / KV write");
     const char* gate = (const char*)m->proj.p + (size_t)Hq * dh * m->esize;
     // causal (query, key) pairs: sum over new tokens of (pos0 + t + 1)
@@ -254,6 +256,11 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
   const long M = (long)B * T;
   const int pos0 = c->len;
   const int dt = cf.dtype;
+  // rotary cos/sin for these positions, shared by every full-attention execution
+  if (m->n_fa > 0 && cf.rotary_dims > 0)
+    CK(prof(m, s, P_FA_PREP, 1, 0, 8.0 * T * (cf.rotary_dims / 2),
+            [&] { return rope_table((float2*)m->rope.p, T, pos0, cf.rotary_dims, cf.rope_base, s); }),
+       "rotary table");
   for (size_t i = 0; i < m->sched.size(); ++i) {
     const ExecRow& r = m->sched[i];
     if (!r.in_loop) {

@@ -52,7 +52,7 @@ struct loop_model {
   size_t esize = 2;
   // activation workspace, sized for `ws_tokens` tokens
   long ws_tokens = 0;
-  DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, gdn_ws, gemm_ws, last;
+  DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, gdn_ws, gemm_ws, rope, last;
   int in_gdn = 0, in_fa = 0;
   Profiler prof;
   DevBuf wrt;                    // [n_layers][8][2d] transposed routing maps (looped layers)
