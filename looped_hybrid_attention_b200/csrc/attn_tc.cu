@@ -1,10 +1,12 @@
 // Causal GQA flash attention on the 5th-generation tensor cores, head dim 256, bf16
 // ("Loop-9B engineering teardown" §三: GQA 16 q / 4 KV heads, head dim 256, output gate).
 //
-// One CTA = 128 query rows of one q head.  Warps:
-//   0     TMA: the Q tile once (4 x [128 x 64] sub-tiles), then K and V tiles of 64 keys
-//         into a 2-stage ring (3-D maps over the per-execution slab, so keys past Tkv
-//         read as zeros);
+// One CTA = 128 MMA rows = the Hq/Hkv q heads of one KV group x 128/(Hq/Hkv) query
+// positions (row r: head r / QT, position q0 + r % QT), so every K/V tile loaded serves
+// all heads that share it.  Warps:
+//   0     TMA: the Q tile once (per head, 4 x [QT x 64] boxes), then K and V tiles of 64
+//         keys into a 2-stage ring (3-D maps over the per-execution slab, so keys past
+//         Tkv read as zeros);
 //   1     MMA: S_j = Q K_j^T (M 128, N 64, K 256) into one of two TMEM buffers, and
 //         O += P_j V_j (M 128, N 256, K 64; V is an MN-major operand) into TMEM;
 //   2..5  softmax, one thread per query row (TMEM lane = row, so the row max and
@@ -12,7 +14,8 @@
 //         the 128-byte-swizzled K-major layout the MMA reads; O is rescaled in TMEM
 //         only when the running max grows by more than 2^8 (the stale max cancels in
 //         the final O / l); finally O / l * sigmoid(gate) is stored.
-// Q K^T of tile j+1 overlaps the softmax of tile j.  All waits are bounded.
+// Q K^T of tile j+1 overlaps the softmax of tile j, and with two P buffers the softmax
+// of tile j+1 overlaps the P.V of tile j.  All waits are bounded.
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -23,21 +26,21 @@ constexpr int AT_M = 128, AT_N = 64, AT_D = 256;
 constexpr int Q_BYTES = AT_M * AT_D * 2;         // 64 KiB
 constexpr int KV_TILE = AT_N * AT_D * 2;         // 32 KiB each for K and V
 constexpr int P_BYTES = AT_M * AT_N * 2;         // 16 KiB
-constexpr int AT_SMEM = Q_BYTES + 2 * 2 * KV_TILE + P_BYTES + 1024 + 256;
+constexpr int AT_SMEM = Q_BYTES + 2 * 2 * KV_TILE + 2 * P_BYTES + 1024 + 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units
 
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tK,
                    const __grid_constant__ CUtensorMap tV, const __nv_bfloat16* __restrict__ gate, int ld_gate,
                    __nv_bfloat16* __restrict__ out, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
-                   float scale_log2) {
+                   float scale_log2, int QT) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + Q_BYTES;                      // stage s: K at s*2*KV_TILE, V at +KV_TILE
-  uint8_t* sP = sKV + 4 * KV_TILE;
-  uint64_t* bars = (uint64_t*)(sP + P_BYTES);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 12);
+  uint8_t* sP = sKV + 4 * KV_TILE;                   // two P buffers (tile j uses j & 1)
+  uint64_t* bars = (uint64_t*)(sP + 2 * P_BYTES);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0;
@@ -45,16 +48,18 @@ __global__ void __launch_bounds__(192, 1)
   auto kv_empty = [&](int s) { return bar0 + 8u * (3 + s); };
   auto s_full = [&](int b) { return bar0 + 8u * (5 + b); };
   auto s_free = [&](int b) { return bar0 + 8u * (7 + b); };
-  const uint32_t p_full = bar0 + 8u * 9, pv_done = bar0 + 8u * 10;
+  // one p_full / pv_done per P buffer, so no barrier runs two phases ahead of its waiter
+  auto p_full = [&](int s) { return bar0 + 8u * (9 + s); };
+  auto pv_done = [&](int s) { return bar0 + 8u * (11 + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = gridDim.x;
   const int qt = n_qt - 1 - blockIdx.x;               // longest causal rows first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kvh = h / (Hq / Hkv);
-  const int q0 = qt * AT_M;
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int rep = Hq / Hkv;
+  const int q0 = qt * QT;
   int k_end = Tkv;
-  if (causal) k_end = min(k_end, q_off + q0 + AT_M);
+  if (causal) k_end = min(k_end, q_off + q0 + QT);
   const int n_kv = (k_end + AT_N - 1) / AT_N;
 
   if (threadIdx.x == 0) {
@@ -65,8 +70,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(s_full(s), 1);
       mbar_init(s_free(s), 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(p_full(s), 128);
+      mbar_init(pv_done(s), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -85,8 +92,11 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       mbar_expect_tx(q_full, Q_BYTES);
+      for (int hh = 0; hh < rep; ++hh)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tma_load_3d(smem_u32(sQ + c * (Q_BYTES / 4)), &tQ, q_full, h * AT_D + c * 64, q0, b);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(smem_u32(sQ + c * (Q_BYTES / 4) + hh * QT * 128), &tQ, q_full, (kvh * rep + hh) * AT_D + c * 64,
+                      q0, b);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j & 1;
         if (!mbar_wait(kv_empty(s), ((j >> 1) & 1) ^ 1, abort_flag)) goto done;
@@ -123,23 +133,25 @@ __global__ void __launch_bounds__(192, 1)
       if (n_kv > 0 && !issue_qk(0)) goto done;
       for (int j = 0; j < n_kv; ++j) {
         if (j + 1 < n_kv && !issue_qk(j + 1)) goto done;
-        if (!mbar_wait(p_full, j & 1, abort_flag)) goto done;
+        if (!mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag)) goto done;
         fence_after();
-        const uint32_t pa = smem_u32(sP);
+        const uint32_t pa = smem_u32(sP + (j & 1) * P_BYTES);
         const uint32_t va = smem_u32(sKV + (j & 1) * 2 * KV_TILE + KV_TILE);
 #pragma unroll
         for (int ks = 0; ks < AT_N / 16; ++ks)
           mma_bf16(tO, sw128_desc(pa + ks * 32), sw128_desc_mn(va + ks * 2048, KV_TILE / 4), id_pv,
                    (j > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(pv_done);
+        mma_commit(pv_done(j & 1));
         mma_commit(kv_empty(j & 1));
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;                // query row within the tile
-    const int qpos = q_off + q0 + r;
+    const int r = quarter * 32 + lane;                // MMA row: head r / QT, query q0 + r % QT
+    const int qi = r % QT;
+    const int h = kvh * rep + r / QT;
+    const int qpos = q_off + q0 + qi;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < n_kv; ++j) {
@@ -163,9 +175,9 @@ __global__ void __launch_bounds__(192, 1)
         t[i] = ok ? raw * scale_log2 : -INFINITY;
         mt = fmaxf(mt, t[i]);
       }
-      if (j > 0 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag)) goto done;
       if (mt > m_used + RESCALE_THRESHOLD) {
         if (j > 0) {                                  // O holds tiles < j scaled by 2^-m_used
+          if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) goto done;
           const float corr = exp2f(m_used - mt);
           l *= corr;
           fence_after();
@@ -182,10 +194,12 @@ __global__ void __launch_bounds__(192, 1)
         }
         m_used = mt;
       }
+      // P buffer j & 1 was last read by the P.V of tile j - 2
+      if (j >= 2 && !mbar_wait(pv_done(j & 1), ((j >> 1) & 1) ^ 1, abort_flag)) goto done;
       // P row (bf16) into the swizzled [128 x 64] K-major tile: 16-byte chunk c of row r
       // sits at chunk position c ^ (r & 7)
       float psum = 0.f;
-      uint8_t* prow = sP + r * 128;
+      uint8_t* prow = sP + (j & 1) * P_BYTES + r * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t w[4];
@@ -201,11 +215,11 @@ __global__ void __launch_bounds__(192, 1)
       l += psum;
       fence_proxy_async();
       fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(j & 1));
     }
-    if (n_kv > 0 && !mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag)) goto done;
+    if (n_kv > 0 && !mbar_wait(pv_done((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1, abort_flag)) goto done;
     fence_after();
-    const int row = q0 + r;
+    const int row = q0 + qi;
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
     for (int c = 0; c < AT_D / 32; ++c) {
@@ -253,8 +267,12 @@ cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, i
                         int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
                         cudaStream_t s) {
   using namespace tc;
+  const int rep = Hq / Hkv;
+  if (rep < 1 || AT_M % rep != 0) return cudaErrorNotSupported;
+  const int QT = AT_M / rep;                              // query positions per CTA
+  if (QT % 8 != 0) return cudaErrorNotSupported;          // whole 8-row swizzle atoms per head
   CUtensorMap mQ, mK, mV;
-  if (!make_map_3d(&mQ, q, (long)Hq * AT_D, Tq, B, ld_q, (long)Tq * ld_q, 64, AT_M)) return cudaErrorNotSupported;
+  if (!make_map_3d(&mQ, q, (long)Hq * AT_D, Tq, B, ld_q, (long)Tq * ld_q, 64, QT)) return cudaErrorNotSupported;
   if (!make_map_3d(&mK, k, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
   if (!make_map_3d(&mV, v, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
   static bool attr = false;
@@ -263,10 +281,10 @@ cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, i
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid((Tq + AT_M - 1) / AT_M, Hq, B);
+  dim3 grid((Tq + QT - 1) / QT, Hkv, B);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)AT_D);
   attn_tc_kernel<<<grid, 192, AT_SMEM, s>>>(mQ, mK, mV, (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, Tq,
-                                            Tkv, q_off, Hq, Hkv, causal, scale_log2);
+                                            Tkv, q_off, Hq, Hkv, causal, scale_log2, QT);
   return cudaGetLastError();
 }
 

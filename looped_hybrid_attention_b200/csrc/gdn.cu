@@ -264,7 +264,7 @@ struct GdnWsB {
 };
 
 template <typename T, int DK, int DV, bool WB>
-__global__ void __launch_bounds__(256) gdn_intra_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ g,
                                                         const float* __restrict__ beta, float* __restrict__ ws,
                                                         int T_len, int H, int n_chunks) {
