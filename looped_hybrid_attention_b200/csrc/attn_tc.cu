@@ -29,6 +29,13 @@ constexpr int P_BYTES = AT_M * AT_N * 2;         // 16 KiB
 constexpr int AT_SMEM = Q_BYTES + 2 * 2 * KV_TILE + 2 * P_BYTES + 1024 + 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units
 
+// 2^x as one MUFU op (x <= 0 here after the row-max shift; denormal results flush to 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tK,
                    const __grid_constant__ CUtensorMap tV, const __nv_bfloat16* __restrict__ gate, int ld_gate,
@@ -164,17 +171,28 @@ __global__ void __launch_bounds__(192, 1)
       tmem_wait_ld();
       fence_before();
       mbar_arrive(s_free(s));
+      // raw scores; the max is taken before scaling (scale > 0).  Only tiles that reach
+      // the causal diagonal or the end of the keys need the per-element mask.
       float t[64];
-      float mt = -INFINITY;
+      float mr = -INFINITY;
       const int kbase = j * AT_N;
+      const bool all_visible = kbase + AT_N <= Tkv && (!causal || kbase + AT_N - 1 <= q_off + q0);
+      if (all_visible) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float raw = __uint_as_float(i < 32 ? sa[i] : sb[i - 32]);
-        const int key = kbase + i;
-        const bool ok = key < Tkv && (!causal || key <= qpos);
-        t[i] = ok ? raw * scale_log2 : -INFINITY;
-        mt = fmaxf(mt, t[i]);
+        for (int i = 0; i < 64; ++i) {
+          t[i] = __uint_as_float(i < 32 ? sa[i] : sb[i - 32]);
+          mr = fmaxf(mr, t[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int key = kbase + i;
+          const bool ok = key < Tkv && (!causal || key <= qpos);
+          t[i] = ok ? __uint_as_float(i < 32 ? sa[i] : sb[i - 32]) : -INFINITY;
+          mr = fmaxf(mr, t[i]);
+        }
       }
+      const float mt = mr * scale_log2;
       if (mt > m_used + RESCALE_THRESHOLD) {
         if (j > 0) {                                  // O holds tiles < j scaled by 2^-m_used
           if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) goto done;
@@ -205,9 +223,10 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(t[c * 8 + 2 * e] - m_used), exp2f(t[c * 8 + 2 * e + 1] - m_used));
-          const float2 back = __bfloat1622float2(pr);
-          psum += back.x + back.y;
+          const float p0 = ex2(fmaf(t[c * 8 + 2 * e], scale_log2, -m_used));
+          const float p1 = ex2(fmaf(t[c * 8 + 2 * e + 1], scale_log2, -m_used));
+          psum += p0 + p1;
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           w[e] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
