@@ -56,6 +56,18 @@ __global__ void __launch_bounds__(192, 1)
   const int n_units = n_tiles * splits;
   const int kps = (kb_n + splits - 1) / splits;
   auto unit_tile = [&](int u) { return u % n_tiles; };
+  // Tile t -> (m-block, n-block), grouped GROUP_M m-blocks at a time: a wave of CTAs
+  // covers a compact block of outputs, so the activation rows of a group stay in L2
+  // while every weight column streams past them once per group.
+  constexpr int GROUP_M = 16;
+  auto tile_mn = [&](int t, int& m0, int& n0) {
+    const int per_group = GROUP_M * nb;
+    const int grp = t / per_group, first_m = grp * GROUP_M;
+    const int gm = min(GROUP_M, mb - first_m);
+    const int in = t % per_group;
+    m0 = (first_m + in % gm) * BM;
+    n0 = (in / gm) * OUT_COLS;
+  };
   auto unit_kb0 = [&](int u) { return (u / n_tiles) * kps; };
   auto unit_kb1 = [&](int u) { return min(kb_n, (u / n_tiles + 1) * kps); };
   const uint32_t bar0 = smem_u32(bars);
@@ -98,7 +110,8 @@ __global__ void __launch_bounds__(192, 1)
       int it = 0;
       for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
         const int t = unit_tile(u);
-        const int m0 = (t % mb) * BM, n0 = (t / mb) * OUT_COLS;
+        int m0, n0;
+        tile_mn(t, m0, n0);
         for (int kb = unit_kb0(u); kb < unit_kb1(u); ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag)) goto done;
@@ -148,7 +161,8 @@ __global__ void __launch_bounds__(192, 1)
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
       const int t = unit_tile(u);
-      const int m0 = (t % mb) * BM, n0 = (t / mb) * OUT_COLS;
+      int m0, n0;
+        tile_mn(t, m0, n0);
       if (!mbar_wait(tfull_bar(acc), (local >> 1) & 1, abort_flag)) goto done;
       fence_after();
       const int row = m0 + quarter * 32 + lane;
