@@ -185,6 +185,22 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
+    kernel's sources have changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = b"".join(open(os.path.join(ROOT, "looped_hybrid_attention_b200", "csrc", n), "rb").read()
+                   for n in ("gemm_tc.cu", "tc_common.cuh"))
+    if hashlib.sha256(src).hexdigest() != rec.get("kernel_sources_sha256"):
+        return None
+    return rec.get("traffic_bytes_per_launch_step_average")
+
+
 def summarize(kernels, steps, peaks, sustained=True, tensor_bound=("gemm", "attention", "gdn_chunk")):
     """Roofline entry for the dominant kernel class and a per-class table.
 
@@ -204,7 +220,7 @@ def summarize(kernels, steps, peaks, sustained=True, tensor_bound=("gemm", "atte
     roof.update({"kernel": name, "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "launches": k["launches"], "ms_per_launch": round(k["ms"] / k["launches"], 4),
                  "algorithmic_per_launch": (k["flops"] if roof["bound"] == "tensor" else k["bytes"]) / k["launches"],
-                 "traffic": None})
+                 "traffic": recorded_traffic(name) if name == "gemm" and tensor_bound else None})
     per_kernel = {}
     total_ms = sum(v["ms"] for v in kernels.values())
     for kname, v in sorted(kernels.items(), key=lambda kv: -kv[1]["ms"]):
