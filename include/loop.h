@@ -248,7 +248,9 @@ loop_status fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
  * Modes 0-2 then route from X': l = RMSNorm(flatten X') W_r + b_r (fp32, no gain),
  * H_pre = sigmoid(l[0:2]), H_post = 2 sigmoid(l[2:4]), H_res = Sinkhorn_iters(exp(l[4:8])),
  * write X_out [N, 2, d], x_in [N, d] = sum_s H_pre[s] X'_s, and coeffs_out [N, 8].
- * Routing reads X' as stored (rounded to dtype). */
+ * Routing reads X' as stored (rounded to dtype).  X_out may equal X_in (in-place MIX).
+ * Every array pointer must be 16-byte aligned (LOOP_ERR_INVALID_ARG otherwise); d must
+ * be a multiple of 8. */
 loop_status mhc_route_mix(int mode, const void* X_in, const void* F, const float* coeffs_in,
                           const float* w_r, const float* b_r, void* X_out, void* x_in,
                           void* h_out, float* coeffs_out, int N, int d, float eps, int iters,

@@ -312,6 +312,9 @@ loop_status mhc_route_mix(int mode, const void* X_in, const void* F, const float
   if (mode == MHC_MERGE) REQUIRE(h_out, LOOP_ERR_INVALID_ARG, "MERGE needs h_out");
   if (mode != MHC_MERGE) REQUIRE(w_r && b_r && x_in && coeffs_out, LOOP_ERR_INVALID_ARG, "routing needs w_r, b_r, x_in, coeffs_out");
   if (mode == MHC_OPEN || mode == MHC_MIX) REQUIRE(X_out, LOOP_ERR_INVALID_ARG, "OPEN/MIX need X_out");
+  const void* ptrs[] = {X_in, F, coeffs_in, X_out, x_in, h_out, coeffs_out};
+  for (const void* p : ptrs)
+    REQUIRE(((uintptr_t)p & 15) == 0, LOOP_ERR_INVALID_ARG, "mhc_route_mix: array pointers must be 16-byte aligned");
   return launched(mhc(mode, X_in, F, coeffs_in, w_r, b_r, X_out, x_in, h_out, coeffs_out, N, d, eps, iters, dtype,
                       S(stream)),
                   "mhc_route_mix");

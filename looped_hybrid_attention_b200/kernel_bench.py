@@ -5,6 +5,7 @@
   python -m looped_hybrid_attention_b200.kernel_bench attn --T 8192
   python -m looped_hybrid_attention_b200.kernel_bench mhc --T 8192
   python -m looped_hybrid_attention_b200.kernel_bench decode --B 16 --T 32768
+  python -m looped_hybrid_attention_b200.kernel_bench group --T 8192   (one full-width layer group in the model flow)
 
 Inputs are random bf16 tensors created on the device (larger than L2 at the default
 sizes); the printed rate uses the same algorithmic flop/byte counts as bench.py.
@@ -34,7 +35,7 @@ def timed(fn, warmup, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemm", "gdn", "attn", "decode", "mhc"])
+    ap.add_argument("op", choices=["gemm", "gdn", "attn", "decode", "mhc", "group"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
@@ -90,6 +91,25 @@ def main():
         ms = timed(lambda: L.gqa_attn(q, Hq * dh, K, V, T, gate, Hq * dh, out, B, 1, T, T - 1, Hq, Hkv, dh, True, ws),
                    a.warmup, a.iters)
         res.update(shape=[B, T, Hq, Hkv, dh], ms=ms, gbs=B * Hkv * T * dh * 2 * 2 / ms / 1e6)
+    elif a.op == "group":
+        import synth
+        shape = synth.GROUP
+        w = synth.make_weights(shape, seed=0, device=dev)
+        m = L.Model(shape, w)
+        c = m.cache(a.B, a.T)
+        h = torch.randn((a.B, a.T, shape.d), device=dev, generator=g).to(bf)
+        out = torch.empty_like(h)
+
+        def run():
+            c.reset()
+            m.forward_hidden(c, h, out)
+        ms = timed(run, a.warmup, a.iters)
+        m.profile(True)
+        run()
+        torch.cuda.synchronize()
+        prof = {k: [v["launches"], round(v["ms"], 4)] for k, v in m.profile_read().items() if v["launches"]}
+        m.profile(False)
+        res.update(shape=[a.B, a.T], ms=ms, tokens_per_s=a.B * a.T / ms * 1e3, per_kernel_ms=prof)
     else:
         N, d = a.B * a.T, 4096
         X, F = r(N, 2, d), r(N, d)
@@ -100,7 +120,11 @@ def main():
         x_in = torch.empty((N, d), device=dev, dtype=bf)
         ms = timed(lambda: L.mhc_route_mix(L.MHC_MIX, X, F, c_in, w_r, b_r, X, x_in, None, c_out, N, d, 1e-6, 20,
                                            L.BF16), a.warmup, a.iters)
-        res.update(shape=[N, d], ms=ms, gbs=N * (2 * 6 * d + 64) / ms / 1e6)
+        h = torch.empty((N, d), device=dev, dtype=bf)
+        ms_m = timed(lambda: L.mhc_route_mix(L.MHC_MERGE, X, F, c_in, None, None, None, None, h, None, N, d, 1e-6, 20,
+                                             L.BF16), a.warmup, a.iters)
+        res.update(shape=[N, d], ms=ms, gbs=N * (2 * 6 * d + 64) / ms / 1e6,
+                   merge_ms=ms_m, merge_gbs=N * (2 * 4 * d + 32) / ms_m / 1e6)
     assert L.device_error() == 0
     print(json.dumps(res))
 

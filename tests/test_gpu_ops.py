@@ -34,7 +34,7 @@ def test_sinkhorn_fp32(cuda, n):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19), (4096, 1501), (256, 2050)])
+@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19), (4096, 1501), (256, 2050), (1024, 1100), (2048, 1057)])
 def test_mhc_modes(cuda, dtype, d, N):
     import looped_hybrid_attention_b200 as L
     code = L.BF16 if dtype == "bf16" else L.F32
@@ -94,6 +94,26 @@ def test_mhc_zero_routing_is_plain_residual(cuda):
     hm = torch.empty_like(h)
     L.mhc_route_mix(L.MHC_MERGE, X, F, c, None, None, None, None, hm, None, N, d, 1e-6, 20, L.F32)
     assert torch.allclose(hm, h + F, atol=1e-5)
+
+
+@pytest.mark.parametrize("N", [10, 1100])
+def test_mhc_extreme_routing_logits(cuda, N):
+    """Residual logits 95 apart: one row of exp(l - max) sums to a denormal, where a
+    reciprocal-and-multiply normalisation would overflow; the Sinkhorn must still match."""
+    import looped_hybrid_attention_b200 as L
+    d = 256
+    h = rnd((N, d), 11, "hx", dtype="bf16")
+    X = torch.empty((N, 2, d), dtype=torch.bfloat16, device=cuda)
+    x_in = torch.empty((N, d), dtype=torch.bfloat16, device=cuda)
+    c = torch.empty((N, 8), device=cuda)
+    w_r = torch.zeros((2 * d, 8), device=cuda)
+    b_r = torch.tensor([0.0, 0.0, 0.0, 0.0, 0.0, 1.0, -95.0, -95.0], device=cuda)
+    L.mhc_route_mix(L.MHC_OPEN, h, None, None, w_r, b_r, X, x_in, None, c, N, d, 1e-6, 20, L.BF16)
+    pre, post, res = ops.mhc_coeffs(ops.mhc_open(to64(h)), to64(w_r), to64(b_r), 1e-6, 20)
+    got = to64(c)
+    assert np.isfinite(got).all()
+    assert np.abs(got[:, 4:8].reshape(N, 2, 2) - res).max() < 1e-5
+    assert np.abs(got[:, 0:4] - np.concatenate([pre, post], axis=1)).max() < 1e-6
 
 
 # ----------------------------------------------------------------------------- norms, embedding, argmax
