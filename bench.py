@@ -10,6 +10,9 @@ prefill of batch 1 x 8192 uniform random token ids.  One step = one prefill (all
 --gpus N > 1 it runs under torchrun as N independent replicas (the forward pass
 has no exchange step), one process per GPU; time is the max over ranks.
 `--impl reference` times the CPU oracle instead, on a bounded sample.
+
+The same line carries two more legs of the same stack: "decode" (batch 64 over
+32,768-token contexts, 256 greedy steps) and "long_prefill" (batch 1, 131,072 tokens).
 """
 from __future__ import annotations
 
@@ -334,6 +337,55 @@ def run_decode(args, m, s, dev, world, seed):
     return out
 
 
+def run_long(args, m, s, dev, world, seed):
+    """Long-context prefill: batch 1, 131,072 uniform random ids in one call (14 KV slabs of
+    131,072 positions, 42 GDN states).  One step is ~6 s, so this leg runs one warm-up and
+    --long-steps timed steps."""
+    import torch
+
+    import looped_hybrid_attention_b200 as L
+    import synth
+    T = args.long_seq
+    c = m.cache(1, T)
+    ids = synth.uniform_ids((1, T), s.vocab, seed, "long", device=dev)
+    logits = torch.empty((1, s.vocab), device=dev)
+    stream = torch.cuda.current_stream()
+    torch.cuda.reset_peak_memory_stats(dev)
+    c.reset()
+    m.prefill(c, ids, logits, stream)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert torch.isfinite(logits).all(), "non-finite logits"
+    m.profile(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        ev0.record(stream)
+        for _ in range(args.long_steps):
+            c.reset()
+            m.prefill(c, ids, logits, stream)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    kernels = m.profile_read()
+    m.profile(False)
+    free, total = torch.cuda.mem_get_info(dev)
+    kv_bytes, st_bytes = c.nbytes()
+    roof, per_kernel = summarize(kernels, args.long_steps, load_peaks())
+    out = {"metric": "prefill tokens/s (56-execution looped hybrid stack)",
+           "workload": f"9B-shape stack, long-context prefill B=1 T={T}, bf16, random-init weights",
+           "value": round(T * args.long_steps * world / (ms / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(ms / args.long_steps, 1), "steps": args.long_steps, "warmup": 1,
+           "kv_slab_bytes": kv_bytes, "gdn_state_bytes": st_bytes,
+           "device_bytes_in_use": total - free,
+           "gpu_launches": sum(v["launches"] for v in kernels.values()),
+           "roofline": roof, "kernels": per_kernel, "clocks": clk.summary()}
+    del c
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -411,10 +463,13 @@ def run_ours(args, world, rank, local):
                     "h2d_bytes_per_step": ids.numel() * 4, "d2h_bytes_per_step": logits.numel() * 4},
             "gpu_launches": launches, "roofline": roof, "kernels": per_kernel,
             "clocks": clk.summary()}
-    if not args.no_decode:
+    if not args.no_decode or not args.no_long:
         del c
         torch.cuda.empty_cache()
+    if not args.no_decode:
         line["decode"] = run_decode(args, m, s, dev, world, args.seed + rank)
+    if not args.no_long:
+        line["long_prefill"] = run_long(args, m, s, dev, world, args.seed + rank)
     if rank != 0:
         return
     if world == 1 and not args.no_cpu_baseline:
@@ -435,6 +490,9 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=64)
     ap.add_argument("--decode-context", type=int, default=32768)
     ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill measurement")
+    ap.add_argument("--long-seq", type=int, default=131072)
+    ap.add_argument("--long-steps", type=int, default=1)
     ap.add_argument("--decode-real-prefill", action="store_true",
                     help="fill the decode contexts with a real prefill instead of random cache values")
     args = ap.parse_args()

@@ -267,10 +267,15 @@ loop_status sinkhorn_fp32(const float* logits, float* out, int N, int n, int ite
  *   2 SWIGLU: Y [M, N] = silu(X W^T) * (X W2^T), W2 [N, K] (the FFN's up map)
  *   3 F32:    Y [M, N] fp32
  * K must be a multiple of 8 for bf16.
+ * bf16 calls with M <= 128 (decode batches, a last position) stream W through every SM
+ * with the batch as the MMA's N dimension.
  * workspace: optional device scratch of loop_linear_workspace_bytes(M, N, K, epilogue)
- * bytes (NULL = none).  With it, bf16 calls with M <= 128 split K across more CTAs
- * (fp32 partial sums, then a reduction that applies the epilogue); calls sharing a
- * workspace must not overlap on the GPU. */
+ * bytes (NULL = none), ZERO-FILLED by the caller before its first use.  With it, bf16
+ * calls with M <= 128 may split a 128-column tile's K range between CTAs: the parts are
+ * summed there in fp32 and the CTA that completes a tile applies the epilogue and
+ * zero-fills the tile's slice again, so a completed call leaves the workspace as it
+ * found it (a call cut short by a device error may not).  Without it, every tile is
+ * computed whole by one CTA.  Calls sharing a workspace must not overlap on the GPU. */
 loop_status loop_linear(const void* X, int ldx, const void* W, const void* W2, const void* R,
                         int ldr, void* Y, int ldy, int M, int N, int K, int epilogue,
                         void* workspace, int dtype, void* stream);

@@ -35,8 +35,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                    const __grid_constant__ CUtensorMap tB2, void* __restrict__ Y, int ldy,
-                   const __nv_bfloat16* __restrict__ R, int ldr, int M, int N, int K, int vec_ok, int splits,
-                   float* __restrict__ partial) {
+                   const __nv_bfloat16* __restrict__ R, int ldr, int M, int N, int K, int vec_ok) {
   using C = Cfg<BN>;
   constexpr int STAGES = C::STAGES;
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;   // output columns per tile
@@ -52,10 +51,6 @@ __global__ void __launch_bounds__(192, 1)
   const int nb = (N + OUT_COLS - 1) / OUT_COLS;
   const int n_tiles = mb * nb;
   const int kb_n = (K + BK - 1) / BK;
-  // split-K: a work unit is (tile, K-slice); with splits == 1 a unit is a tile
-  const int n_units = n_tiles * splits;
-  const int kps = (kb_n + splits - 1) / splits;
-  auto unit_tile = [&](int u) { return u % n_tiles; };
   // Tile t -> (m-block, n-block), grouped GROUP_M m-blocks at a time: a wave of CTAs
   // covers a compact block of outputs, so the activation rows of a group stay in L2
   // while every weight column streams past them once per group.
@@ -68,8 +63,6 @@ __global__ void __launch_bounds__(192, 1)
     m0 = (first_m + in % gm) * BM;
     n0 = (in / gm) * OUT_COLS;
   };
-  auto unit_kb0 = [&](int u) { return (u / n_tiles) * kps; };
-  auto unit_kb1 = [&](int u) { return min(kb_n, (u / n_tiles + 1) * kps); };
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -108,11 +101,10 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int it = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        const int t = unit_tile(u);
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
         int m0, n0;
         tile_mn(t, m0, n0);
-        for (int kb = unit_kb0(u); kb < unit_kb1(u); ++kb, ++it) {
+        for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag)) goto done;
           const uint32_t a_dst = smem_u32(smem + (size_t)s * C::STAGE_BYTES);
@@ -133,13 +125,12 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BM, BN);
       int it = 0, local = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
         const int acc = local & 1;
         if (!mbar_wait(tempty_bar(acc), ((local >> 1) & 1) ^ 1, abort_flag)) goto done;
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const int kb0 = unit_kb0(u);
-        for (int kb = kb0; kb < unit_kb1(u); ++kb, ++it) {
+        for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(full_bar(s), (it / STAGES) & 1, abort_flag)) goto done;
           fence_after();
@@ -148,7 +139,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16(d_tmem, sw128_desc(a_addr + k * 32), sw128_desc(b_addr + k * 32), idesc,
-                     (kb > kb0 || k > 0) ? 1u : 0u);
+                     (kb > 0 || k > 0) ? 1u : 0u);
           mma_commit(empty_bar(s));          // ring slot is free once these MMAs have read it
         }
         mma_commit(tfull_bar(acc));          // accumulator ready for the epilogue
@@ -158,42 +149,14 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------------------------------------------------------- epilogue (warps 2..5)
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
     int local = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
       const int acc = local & 1;
-      const int t = unit_tile(u);
       int m0, n0;
-        tile_mn(t, m0, n0);
+      tile_mn(t, m0, n0);
       if (!mbar_wait(tfull_bar(acc), (local >> 1) & 1, abort_flag)) goto done;
       fence_after();
       const int row = m0 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      if (splits > 1) {
-        // raw fp32 partial sums of this K-slice -> partial[slice][row][col]; SwiGLU keeps the
-        // gate columns at [0, N) and the up columns at [N, 2N)
-        const int NC = EPI == EPI_SWIGLU ? 2 * N : N;
-        float* pp = partial + ((long)(u / n_tiles) * M + row) * NC;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_row + c * 32, r);
-          tmem_wait_ld();
-          int col0 = n0 + c * 32;
-          if (EPI == EPI_SWIGLU && c >= BN / 64) col0 = N + n0 + (c - BN / 64) * 32;
-          const int lim = (EPI == EPI_SWIGLU && c >= BN / 64) ? 2 * N : N;
-          if (row >= M || col0 >= lim) continue;
-          if (vec_ok && col0 + 32 <= lim) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(pp + col0 + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                                                    __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-          } else {
-            for (int i = 0; i < 32 && col0 + i < lim; ++i) pp[col0 + i] = __uint_as_float(r[i]);
-          }
-        }
-        fence_before();
-        mbar_arrive(tempty_bar(acc));
-        continue;
-      }
 #pragma unroll 1
       for (int c = 0; c < OUT_COLS / 32; ++c) {
         uint32_t r[32];
@@ -262,54 +225,9 @@ done:
   }
 }
 
-// Sum of the split-K partial tiles, then the epilogue.  One thread per 8 outputs.
-template <int EPI>
-__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
-                                     const __nv_bfloat16* __restrict__ R, int ldr, void* __restrict__ Y, int ldy) {
-  const int n8 = (N + 7) / 8;
-  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long)M * n8) return;
-  const int m = (int)(idx / n8), n = (int)(idx % n8) * 8;
-  const int NC = EPI == EPI_SWIGLU ? 2 * N : N;
-  const int cnt = min(8, N - n);
-  float g[8] = {0, 0, 0, 0, 0, 0, 0, 0}, u[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int sp = 0; sp < splits; ++sp) {
-    const float* p = partial + ((long)sp * M + m) * NC;
-    for (int i = 0; i < cnt; ++i) {
-      g[i] += p[n + i];
-      if (EPI == EPI_SWIGLU) u[i] += p[N + n + i];
-    }
-  }
-  for (int i = 0; i < cnt; ++i) {
-    float v = g[i];
-    if (EPI == EPI_SWIGLU) v = v / (1.f + expf(-v)) * u[i];
-    if (EPI == EPI_ADD) v += __bfloat162float(R[(long)m * ldr + n + i]);
-    if (EPI == EPI_F32)
-      reinterpret_cast<float*>(Y)[(long)m * ldy + n + i] = v;
-    else
-      reinterpret_cast<__nv_bfloat16*>(Y)[(long)m * ldy + n + i] = __float2bfloat16(v);
-  }
-}
-
-// K-slices for a GEMM with few output tiles (small M): aim for one unit per SM (more
-// slices only add partial-sum traffic), keep at least 4 K-blocks per slice, and fit
-// the partials in `ws_bytes`.
-static int choose_splits(int M, int N, int K, int epi, size_t ws_bytes) {
-  constexpr int BN = 256;
-  const int out_cols = epi == EPI_SWIGLU ? BN / 2 : BN;
-  const long tiles = (long)((M + BM - 1) / BM) * ((N + out_cols - 1) / out_cols);
-  const int kb = (K + BK - 1) / BK;
-  int sp = (int)((num_sms() + tiles - 1) / tiles);
-  sp = min(sp, kb / 4);
-  sp = min(sp, 16);
-  const long nc = epi == EPI_SWIGLU ? 2L * N : N;
-  while (sp > 1 && (size_t)sp * M * nc * 4 > ws_bytes) --sp;
-  return sp < 1 ? 1 : sp;
-}
-
 template <int BN, int EPI>
 static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y,
-                          int ldy, int M, int N, int K, cudaStream_t s, void* ws, size_t ws_bytes) {
+                          int ldy, int M, int N, int K, cudaStream_t s) {
   using C = Cfg<BN>;
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   constexpr int B_ROWS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
@@ -332,31 +250,17 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
   const int esz = EPI == EPI_F32 ? 4 : 2;
   const int vec_ok = ((ldy * esz) % 16 == 0) && (((uintptr_t)Y) % 16 == 0) &&
                      (EPI != EPI_ADD || ((ldr * 2) % 16 == 0 && ((uintptr_t)R) % 16 == 0));
-  const int splits = (ws && M <= BM) ? choose_splits(M, N, K, EPI, ws_bytes) : 1;
-  const long units = tiles * splits;
-  const int grid2 = (int)(units < num_sms() ? units : num_sms());
-  const int nc = EPI == EPI_SWIGLU ? 2 * N : N;
-  const int vec = splits > 1 ? (nc % 4 == 0 && ((uintptr_t)ws % 16) == 0) : vec_ok;
-  kern<<<grid2, 192, C::SMEM, s>>>(tA, tB, tB2, Y, ldy, (const __nv_bfloat16*)R, ldr, M, N, K, vec, splits,
-                                   (float*)ws);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
-  const long work = (long)M * ((N + 7) / 8);
-  splitk_reduce_kernel<EPI><<<(unsigned)((work + 255) / 256), 256, 0, s>>>((const float*)ws, splits, M, N,
-                                                                          (const __nv_bfloat16*)R, ldr, Y, ldy);
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, 192, C::SMEM, s>>>(tA, tB, tB2, Y, ldy, (const __nv_bfloat16*)R, ldr, M, N, K, vec_ok);
   return cudaGetLastError();
 }
 
 }  // namespace tc
 
-int linear_launches(int M, int N, int K, int epi, const void* ws, size_t ws_bytes) {
-  return (ws && M > 0 && M <= tc::BM && tc::choose_splits(M, N, K, epi, ws_bytes) > 1) ? 2 : 1;
-}
-
 size_t linear_workspace_bytes(int M, int N, int K, int epi) {
-  if (M > tc::BM || M <= 0) return 0;
-  const long nc = epi == EPI_SWIGLU ? 2L * N : N;
-  return (size_t)16 * M * nc * 4;      // up to 16 K-slices
+  (void)K;
+  if (M > tc::BM || M <= 0 || N <= 0) return 0;
+  return linear_skinny_workspace_bytes(M, N, epi);
 }
 
 cudaError_t linear_tc(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y, int ldy,
@@ -365,11 +269,12 @@ cudaError_t linear_tc(const void* X, int ldx, const void* W, const void* W2, con
   // TMA needs 16-byte aligned bases and row strides
   if (((uintptr_t)X) % 16 || ((uintptr_t)W) % 16 || (ldx * 2) % 16 || (K * 2) % 16) return cudaErrorNotSupported;
   if (epi == EPI_SWIGLU && ((uintptr_t)W2) % 16) return cudaErrorNotSupported;
+  if (M <= tc::BM) return linear_skinny(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, s, ws, ws_bytes);
   switch (epi) {
-    case EPI_STORE: return tc::launch<256, EPI_STORE>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s, ws, ws_bytes);
-    case EPI_ADD: return tc::launch<256, EPI_ADD>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s, ws, ws_bytes);
-    case EPI_SWIGLU: return tc::launch<256, EPI_SWIGLU>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s, ws, ws_bytes);
-    case EPI_F32: return tc::launch<256, EPI_F32>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s, ws, ws_bytes);
+    case EPI_STORE: return tc::launch<256, EPI_STORE>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s);
+    case EPI_ADD: return tc::launch<256, EPI_ADD>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s);
+    case EPI_SWIGLU: return tc::launch<256, EPI_SWIGLU>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s);
+    case EPI_F32: return tc::launch<256, EPI_F32>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s);
   }
   return cudaErrorNotSupported;
 }

@@ -17,7 +17,8 @@ cudaError_t embed(const int32_t* ids, const void* E, void* out, int M, int d, in
                   cudaStream_t s);
 cudaError_t argmax(const float* logits, int32_t* next, int B, int V, cudaStream_t s);
 
-// ws / ws_bytes: optional scratch for split-K when M <= 128 (linear_workspace_bytes).
+// ws / ws_bytes: optional zero-filled scratch for M <= 128 (linear_workspace_bytes): tiles
+// split between CTAs are summed there; each call leaves it zero-filled again.
 cudaError_t linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
                    void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s, void* ws = nullptr,
                    size_t ws_bytes = 0);
@@ -26,7 +27,11 @@ cudaError_t linear_tc(const void* X, int ldx, const void* W, const void* W2, con
                       void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s, void* ws = nullptr,
                       size_t ws_bytes = 0);
 size_t linear_workspace_bytes(int M, int N, int K, int epi);
-int linear_launches(int M, int N, int K, int epi, const void* ws, size_t ws_bytes);
+// M <= 128 (decode batches, the last prefill position): weight-streaming tcgen05 kernel.
+cudaError_t linear_skinny(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
+                          void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s, void* ws,
+                          size_t ws_bytes);
+size_t linear_skinny_workspace_bytes(int M, int N, int epi);
 cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, const void* R,
                         int ldr, void* Y, int ldy, int M, int N, int K, int epi, int dtype,
                         cudaStream_t s);

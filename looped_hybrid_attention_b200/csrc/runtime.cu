@@ -101,8 +101,14 @@ std::vector<ExecRow> build_schedule(const loop_config& c) {
   return rows;
 }
 
+#define CK(call, what)                                  \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);  \
+  } while (0)
+
 // ------------------------------------------------------------------ workspace
-static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tkv_max) {
+static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tkv_max, cudaStream_t s) {
   const loop_config& c = m->cfg;
   const size_t es = m->esize;
   const int d = c.d;
@@ -129,25 +135,28 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->rope, (size_t)Tq * (c.rotary_dims / 2) * sizeof(float2)},
       {&m->attn_ws, gqa_workspace_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_head_dim)},
       {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
-      // split-K partials for projections with few tokens (the widest: the FFN gate/up pair)
-      {&m->gemm_ws, M <= 128 ? linear_workspace_bytes((int)M, std::max(c.ffn, std::max(m->in_fa, m->in_gdn)), c.d,
-                                                      EPI_SWIGLU)
-                             : 0},
       {&m->last, (size_t)B * d * es},
   };
   for (auto& n : need) {
     cudaError_t e = n.b->ensure(n.bytes < 256 ? 256 : n.bytes);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
   }
+  // partial sums of projections with few rows (<= 128): the layer projections of these
+  // tokens and the LM head on each sequence's last position; zero-filled once, and every
+  // projection leaves it zero-filled
+  size_t gws = 0;
+  if (M <= 128) {
+    const int ns[4][2] = {{m->in_gdn, EPI_STORE}, {m->in_fa, EPI_STORE}, {d, EPI_ADD}, {c.ffn, EPI_SWIGLU}};
+    for (auto& n : ns) gws = std::max(gws, linear_workspace_bytes((int)M, n[0], d, n[1]));
+  }
+  if (B <= 128) gws = std::max(gws, linear_workspace_bytes(B, c.vocab, d, EPI_F32));
+  if (gws > m->gemm_ws.bytes) {
+    CK(m->gemm_ws.ensure(gws), "projection workspace allocation");
+    CK(cudaMemsetAsync(m->gemm_ws.p, 0, m->gemm_ws.bytes, s), "projection workspace zero fill");
+  }
   if (M > m->ws_tokens) m->ws_tokens = M;
   return LOOP_OK;
 }
-
-#define CK(call, what)                                  \
-  do {                                                  \
-    cudaError_t e_ = (call);                            \
-    if (e_ != cudaSuccess) return cuda_fail(e_, what);  \
-  } while (0)
 
 // ------------------------------------------------------------------ one decoder layer
 // x [M, d] -> writes the layer's result: plain layers h = x + F (into `h_out`),
@@ -160,17 +169,13 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
   const int d = cf.d, dt = cf.dtype;
   const double es = (double)m->esize;
   double fl, by;
-  // kernel launches of one projection (2 when split-K adds its reduction)
-  auto gl = [&](long Mm, int N, int K, int epi) {
-    return cf.dtype == LOOP_BF16 ? linear_launches((int)Mm, N, K, epi, m->gemm_ws.p, m->gemm_ws.bytes) : 1;
-  };
   CK(prof(m, s, P_RMSNORM, 1, 0, es * (2.0 * M * d + d),
           [&] { return rmsnorm(x, nullptr, nullptr, w.attn_norm, m->xn.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (mixer)");
   if (r.kind == 0) {
     const int H = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
     gemm_work(M, m->in_gdn, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, gl(M, m->in_gdn, d, EPI_STORE), fl, by,
+    CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d,
                                 EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "GDN input projection");
@@ -198,14 +203,14 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
          "GDN chunked scan");
     }
     gemm_work(M, d, H * dv, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, gl(M, d, H * dv, EPI_STORE), fl, by,
+    CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->o.p, H * dv, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, H * dv, EPI_STORE,
                                 dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "GDN output projection");
   } else {
     const int Hq = cf.fa_q_heads, Hkv = cf.fa_kv_heads, dh = cf.fa_head_dim;
     gemm_work(M, m->in_fa, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, gl(M, m->in_fa, d, EPI_STORE), fl, by,
+    CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d,
                                 EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "FA input projection");
@@ -225,7 +230,7 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
                                       pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s); }),
        "GQA attention");
     gemm_work(M, d, Hq * dh, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, gl(M, d, Hq * dh, EPI_STORE), fl, by,
+    CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->o.p, Hq * dh, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, Hq * dh,
                                 EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "FA output projection");
@@ -235,14 +240,14 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
           [&] { return rmsnorm(x, m->mix.p, m->u.p, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (FFN)");
   gemm_work(M, cf.ffn, d, EPI_SWIGLU, m->esize, fl, by);
-  CK(prof(m, s, P_GEMM, gl(M, cf.ffn, d, EPI_SWIGLU), fl, by,
+  CK(prof(m, s, P_GEMM, 1, fl, by,
           [&] { return linear(m->un.p, d, w.w_gate, w.w_up, nullptr, 0, m->act.p, cf.ffn, (int)M, cf.ffn, d, EPI_SWIGLU,
                               dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
      "FFN gate/up (SwiGLU)");
   gemm_work(M, d, cf.ffn, EPI_ADD, m->esize, fl, by);
   const void* res = r.in_loop ? m->mix.p : m->u.p;
   void* dst = r.in_loop ? m->F.p : h_out;
-  CK(prof(m, s, P_GEMM, gl(M, d, cf.ffn, EPI_ADD), fl, by,
+  CK(prof(m, s, P_GEMM, 1, fl, by,
           [&] { return linear(m->act.p, cf.ffn, w.w_down, nullptr, res, d, dst, d, (int)M, d, cf.ffn, EPI_ADD, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
      "FFN down (+ residual)");
   return LOOP_OK;
@@ -318,7 +323,7 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
                         float* logits_last, int B, int T, cudaStream_t s) {
   const loop_config& cf = m->cfg;
   const long M = (long)B * T;
-  loop_status st = ensure_workspace(m, M, B, T, c->max_tokens);
+  loop_status st = ensure_workspace(m, M, B, T, c->max_tokens, s);
   if (st != LOOP_OK) return st;
   st = prepare(m, s);
   if (st != LOOP_OK) return st;
@@ -354,7 +359,7 @@ loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* 
                        cudaStream_t s) {
   const loop_config& cf = m->cfg;
   const int B = c->batch;
-  loop_status st = ensure_workspace(m, B, B, 1, c->max_tokens);
+  loop_status st = ensure_workspace(m, B, B, 1, c->max_tokens, s);
   if (st != LOOP_OK) return st;
   st = prepare(m, s);
   if (st != LOOP_OK) return st;

@@ -57,9 +57,14 @@ def main():
         R = r(a.M, a.N) if a.epi == "add" else None
         Y = torch.empty((a.M, a.N), device=dev, dtype=torch.float32 if a.epi == "f32" else bf)
         epi = {"store": L.EPI_STORE, "add": L.EPI_ADD, "swiglu": L.EPI_SWIGLU, "f32": L.EPI_F32}[a.epi]
-        ms = timed(lambda: L.linear(X, W, Y, epi, W2=W2, R=R), a.warmup, a.iters)
-        flops = 2.0 * a.M * a.N * a.K * (2 if a.epi == "swiglu" else 1)
-        res.update(shape=[a.M, a.N, a.K], epi=a.epi, ms=ms, tflops=flops / ms / 1e9)
+        # zero-filled partial-sum workspace for few rows (M <= 128), as the runtime gives it
+        nws = L.linear_workspace_bytes(a.M, a.N, a.K, epi)
+        ws = torch.zeros(nws // 4 + 1, device=dev) if nws else None
+        ms = timed(lambda: L.linear(X, W, Y, epi, W2=W2, R=R, workspace=ws), a.warmup, a.iters)
+        nmat = 2 if a.epi == "swiglu" else 1
+        flops = 2.0 * a.M * a.N * a.K * nmat
+        byts = 2.0 * (a.M * a.K + nmat * a.N * a.K) + Y.element_size() * a.M * a.N * (2 if a.epi == "add" else 1)
+        res.update(shape=[a.M, a.N, a.K], epi=a.epi, ms=ms, tflops=flops / ms / 1e9, gbs=byts / ms / 1e6)
     elif a.op == "gdn":
         B, T, H, dk = a.B, a.T, a.H, 128
         q = torch.nn.functional.normalize(torch.randn(B, T, H, dk, device=dev, generator=g), dim=-1).to(bf)

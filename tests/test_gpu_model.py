@@ -139,3 +139,37 @@ def test_tiny_stack_long_sequence_fp32(cuda):
     m.forward_hidden(c, h.cuda(), out)
     torch.cuda.synchronize()
     assert rel_l2(to64(out), ref) < TOL["fp32"]
+
+
+@pytest.mark.slow
+def test_full_stack_long_context_prefix(cuda):
+    """The full 9B-shape stack (56 executions, bf16) over a 131,072-token input in one call.
+
+    The stack is causal and every kernel's arithmetic for a row depends only on that row's
+    prefix (fixed chunk and tile boundaries), so the first 8,192 output rows must equal,
+    bit for bit, a separate 8,192-token call; the KV slab of every full-attention execution
+    holds 131,072 written positions, and every output is finite."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.FULL
+    T, T0 = 131072, 8192
+    w = synth.make_weights(s, seed=0, device=cuda)
+    gen = torch.Generator(device=cuda).manual_seed(9)
+    h = torch.randn((1, T, s.d), device=cuda, generator=gen).to(torch.bfloat16)
+    m = L.Model(s, w)
+    c = m.cache(1, T)
+    out = torch.empty_like(h)
+    m.forward_hidden(c, h, out)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert c.length == T
+    assert bool(torch.isfinite(out).all())
+    kv_bytes, _ = c.nbytes()
+    assert kv_bytes == 14 * 4096 * T            # 4 KB per token per full-attention execution
+    last_k = L.device_view(c.kv_ptrs(13)[0], (1, s.fa_kv_heads, T, s.fa_head_dim), torch.bfloat16)
+    assert bool((last_k[0, :, -1].abs().sum(dim=-1) > 0).all())   # the last position was written
+    del c
+    c0 = m.cache(1, T0)
+    out0 = torch.empty((1, T0, s.d), dtype=torch.bfloat16, device=cuda)
+    m.forward_hidden(c0, h[:, :T0].contiguous(), out0)
+    torch.cuda.synchronize()
+    assert torch.equal(out[:, :T0], out0)

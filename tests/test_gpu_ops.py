@@ -159,13 +159,16 @@ def test_embed_and_argmax(cuda):
 @pytest.mark.parametrize("split_k", [False, True])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("M,N,K", [(200, 300, 256), (1, 1000, 512), (130, 64, 4096), (64, 4104, 2048),
-                                   (64, 1000, 12288)])
+                                   (64, 1000, 12288), (16, 130, 520), (17, 384, 8), (33, 4000, 4096),
+                                   (100, 200, 1000), (128, 1000, 2048)])
 def test_linear_epilogues(cuda, dtype, M, N, K, split_k):
+    """Every epilogue against fp64; M <= 128 covers each batch-tile width (16/32/64/128 rows),
+    ragged N and K, with the partial-sum workspace (split tiles) and without it (whole tiles)."""
     import looped_hybrid_attention_b200 as L
     ws = None
     if split_k:
         nb = max(L.linear_workspace_bytes(M, N, K, e) for e in (0, 1, 2, 3))
-        ws = torch.empty(max(nb, 16) // 4, device=cuda)
+        ws = torch.zeros(max(nb, 16) // 4, device=cuda)
     X = rnd((M, K), 12, "X", dtype=dtype)
     W = rnd((N, K), 13, "W", std=0.02, dtype=dtype)
     W2 = rnd((N, K), 14, "W2", std=0.02, dtype=dtype)
@@ -181,6 +184,45 @@ def test_linear_epilogues(cuda, dtype, M, N, K, split_k):
     Yf = torch.empty((M, N), dtype=torch.float32, device=cuda)
     L.linear(X, W, Yf, L.EPI_F32, workspace=ws)
     assert rel_l2(to64(Yf), ref) < (1e-5 if dtype == "fp32" else 1e-4)
+    if ws is not None:
+        torch.cuda.synchronize()
+        assert L.device_error() == 0
+        assert int(torch.count_nonzero(ws)) == 0, "a call must leave the workspace zero-filled"
+
+
+# the projections of one decode step at batch 64 (and the LM head): (N, K, epilogue)
+DECODE_GEMMS = [(6176, 4096, "store"), (4096, 2048, "add"), (10240, 4096, "store"), (4096, 4096, "add"),
+                (12288, 4096, "swiglu"), (4096, 12288, "add"), (248320, 4096, "f32")]
+
+
+@pytest.mark.parametrize("N,K,epi", DECODE_GEMMS)
+def test_linear_decode_shapes(cuda, N, K, epi):
+    """bf16 projections at M = 64 (the decode batch) in the full 9B shapes with the runtime's
+    zero-filled workspace, twice in a row (the second call relies on the first leaving the
+    workspace zero-filled); sampled output columns against fp64."""
+    import looped_hybrid_attention_b200 as L
+    M = 64
+    code = {"store": L.EPI_STORE, "add": L.EPI_ADD, "swiglu": L.EPI_SWIGLU, "f32": L.EPI_F32}[epi]
+    gen = lambda seed: torch.Generator(device=cuda).manual_seed(seed)
+    X = torch.randn((M, K), device=cuda, generator=gen(11)).to(torch.bfloat16)
+    W = (0.02 * torch.randn((N, K), device=cuda, generator=gen(12))).to(torch.bfloat16)
+    W2 = (0.02 * torch.randn((N, K), device=cuda, generator=gen(13))).to(torch.bfloat16) if epi == "swiglu" else None
+    R = torch.randn((M, N), device=cuda, generator=gen(14)).to(torch.bfloat16) if epi == "add" else None
+    Y = torch.empty((M, N), device=cuda, dtype=torch.float32 if epi == "f32" else torch.bfloat16)
+    ws = torch.zeros(L.linear_workspace_bytes(M, N, K, code) // 4 + 1, device=cuda)
+    cols = np.unique(np.r_[0:130, N // 2 - 70:N // 2 + 70, N - 130:N])
+    xr = to64(X)
+    ref = ops.linear(xr, to64(W[cols]))
+    if epi == "swiglu":
+        ref = ops.silu(ref) * ops.linear(xr, to64(W2[cols]))
+    if epi == "add":
+        ref = ref + to64(R[:, cols])
+    for _ in range(2):
+        L.linear(X, W, Y, code, W2=W2, R=R, workspace=ws)
+        torch.cuda.synchronize()
+        assert L.device_error() == 0
+        assert rel_l2(to64(Y[:, cols]), ref) < (1e-4 if epi == "f32" else TOL["bf16"])
+        assert int(torch.count_nonzero(ws)) == 0
 
 
 # ----------------------------------------------------------------------------- Gated DeltaNet
@@ -296,6 +338,37 @@ def test_gdn_chunk_full_length_sampled_heads(cuda):
         assert rel_l2(to64(S[0, sl]), S_ref) < TOL["bf16"]
 
 
+
+@pytest.mark.slow
+def test_gdn_chunk_long_context(cuda):
+    """The long-context prefill shape (T = 131,072, 16 heads x 128, bf16): 2,048 chunks carried
+    through one state; head 7's outputs and final state against the token recurrence."""
+    import looped_hybrid_attention_b200 as L
+    B, T, H, dk = 1, 131072, 16, 128
+    gen = torch.Generator(device=cuda).manual_seed(78)
+    q = torch.nn.functional.normalize(torch.randn(B, T, H, dk, device=cuda, generator=gen), dim=-1).to(torch.bfloat16)
+    k = torch.nn.functional.normalize(torch.randn(B, T, H, dk, device=cuda, generator=gen), dim=-1).to(torch.bfloat16)
+    v = torch.randn(B, T, H, dk, device=cuda, generator=gen).to(torch.bfloat16)
+    # decays near 1 keep the state's memory long (the regime where position errors would show)
+    g = -torch.nn.functional.softplus(torch.randn(B, T, H, device=cuda, generator=gen) - 5.0)
+    beta = torch.sigmoid(torch.randn(B, T, H, device=cuda, generator=gen))
+    S = 0.1 * torch.randn(B, H, dk, dk, device=cuda, generator=gen)
+    S0 = S.clone()
+    out = torch.empty_like(v)
+    scale = 1.0 / np.sqrt(dk)
+    ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=cuda)
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    sl = slice(7, 8)
+    o_ref, S_ref = ops.gdn_recurrent(to64(q[0, :, sl]), to64(k[0, :, sl]), to64(v[0, :, sl]), to64(g[0, :, sl]),
+                                     to64(beta[0, :, sl]), to64(S0[0, sl]), scale)
+    got = to64(out[0, :, sl])
+    assert rel_l2(got, o_ref) < TOL["bf16"]
+    assert rel_l2(got[-4096:], o_ref[-4096:]) < TOL["bf16"]      # the last chunks on their own
+    assert rel_l2(to64(S[0, sl]), S_ref) < TOL["bf16"]
+
+
 # ----------------------------------------------------------------------------- attention
 
 def _fa_case(B, T, Hq, Hkv, dh, dtype, seed):
@@ -393,6 +466,28 @@ def test_attention_full_length_sampled_rows(cuda):
     L.gqa_attn(q, Hq * dh, Kc, Vc, T, None, 0, out, 1, T, T, 0, Hq, Hkv, dh, True)
     rows = np.array([0, 1, 63, 64, 127, 128, 4095, 5000, 8190, 8191])
     ref = ops.attention(to64(q[rows]), to64(Kc[0]).transpose(1, 0, 2), to64(Vc[0]).transpose(1, 0, 2), rows)
+    assert rel_l2(to64(out[rows]).reshape(len(rows), Hq, dh), ref) < TOL["bf16"]
+
+
+
+@pytest.mark.slow
+def test_attention_long_context_sampled_rows(cuda):
+    """The long-context prefill shape (T = 131,072, 16q/4kv x 256, bf16, gate fused): sampled
+    query rows, including the last, against brute-force softmax over their causal prefix."""
+    import looped_hybrid_attention_b200 as L
+    T, Hq, Hkv, dh = 131072, 16, 4, 256
+    gen = torch.Generator(device=cuda).manual_seed(53)
+    q = torch.randn((T, Hq, dh), device=cuda, generator=gen).to(torch.bfloat16)
+    Kc = torch.randn((1, Hkv, T, dh), device=cuda, generator=gen).to(torch.bfloat16)
+    Vc = torch.randn((1, Hkv, T, dh), device=cuda, generator=gen).to(torch.bfloat16)
+    gate = torch.randn((T, Hq * dh), device=cuda, generator=gen).to(torch.bfloat16)
+    out = torch.empty((T, Hq * dh), dtype=torch.bfloat16, device=cuda)
+    L.gqa_attn(q, Hq * dh, Kc, Vc, T, gate, Hq * dh, out, 1, T, T, 0, Hq, Hkv, dh, True)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    rows = np.array([0, 63, 64, 65535, 65536, 100000, 131007, 131008, 131070, 131071])
+    ref = ops.attention(to64(q[rows]), to64(Kc[0]).transpose(1, 0, 2), to64(Vc[0]).transpose(1, 0, 2), rows)
+    ref = ref * ops.sigmoid(to64(gate[rows]).reshape(len(rows), Hq, dh))
     assert rel_l2(to64(out[rows]).reshape(len(rows), Hq, dh), ref) < TOL["bf16"]
 
 
