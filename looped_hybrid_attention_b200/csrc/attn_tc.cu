@@ -5,8 +5,10 @@
 // positions (row r: head r / QT, position q0 + r % QT), so every K/V tile loaded serves
 // all heads that share it.  Warps:
 //   0     TMA: the Q tile once (per head, 4 x [QT x 64] boxes), then K and V tiles of 64
-//         keys into a 2-stage ring (3-D maps over the per-execution slab, so keys past
-//         Tkv read as zeros);
+//         keys into two separate 2-stage rings (3-D maps over the per-execution slab, so
+//         keys past Tkv read as zeros).  A K slot is free as soon as Q K^T has read it,
+//         a V slot once P V has: K tiles stream in about a tile ahead of their use
+//         instead of waiting for the previous P V;
 //   1     MMA: S_j = Q K_j^T (M 128, N 64, K 256) into one of two TMEM buffers, and
 //         O += P_j V_j (M 128, N 256, K 64; V is an MN-major operand) into TMEM;
 //   2..5  softmax, one thread per query row (TMEM lane = row, so the row max and
@@ -44,20 +46,23 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + Q_BYTES;                      // stage s: K at s*2*KV_TILE, V at +KV_TILE
-  uint8_t* sP = sKV + 4 * KV_TILE;                   // two P buffers (tile j uses j & 1)
+  uint8_t* sK = smem + Q_BYTES;                       // K ring: stage s at s * KV_TILE
+  uint8_t* sV = sK + 2 * KV_TILE;                     // V ring
+  uint8_t* sP = sV + 2 * KV_TILE;                     // two P buffers (tile j uses j & 1)
   uint64_t* bars = (uint64_t*)(sP + 2 * P_BYTES);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0;
-  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (5 + b); };
-  auto s_free = [&](int b) { return bar0 + 8u * (7 + b); };
+  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bar0 + 8u * (3 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (5 + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (9 + b); };
+  auto s_free = [&](int b) { return bar0 + 8u * (11 + b); };
   // one p_full / pv_done per P buffer, so no barrier runs two phases ahead of its waiter
-  auto p_full = [&](int s) { return bar0 + 8u * (9 + s); };
-  auto pv_done = [&](int s) { return bar0 + 8u * (11 + s); };
+  auto p_full = [&](int s) { return bar0 + 8u * (13 + s); };
+  auto pv_done = [&](int s) { return bar0 + 8u * (15 + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = gridDim.x;
@@ -72,8 +77,10 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
       mbar_init(s_full(s), 1);
       mbar_init(s_free(s), 128);
     }
@@ -106,14 +113,16 @@ __global__ void __launch_bounds__(192, 1)
                       q0, b);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(kv_empty(s), ((j >> 1) & 1) ^ 1, abort_flag)) goto done;
-        mbar_expect_tx(kv_full(s), 2 * KV_TILE);
-        const uint32_t kd = smem_u32(sKV + s * 2 * KV_TILE), vd = kd + KV_TILE;
+        const uint32_t par = ((j >> 1) & 1) ^ 1;
+        if (!mbar_wait(k_empty(s), par, abort_flag)) goto done;
+        mbar_expect_tx(k_full(s), KV_TILE);
+        const uint32_t kd = smem_u32(sK + s * KV_TILE), vd = smem_u32(sV + s * KV_TILE);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tma_load_3d(kd + c * (KV_TILE / 4), &tK, kv_full(s), c * 64, j * AT_N, b * Hkv + kvh);
-          tma_load_3d(vd + c * (KV_TILE / 4), &tV, kv_full(s), c * 64, j * AT_N, b * Hkv + kvh);
-        }
+        for (int c = 0; c < 4; ++c) tma_load_3d(kd + c * (KV_TILE / 4), &tK, k_full(s), c * 64, j * AT_N, b * Hkv + kvh);
+        if (!mbar_wait(v_empty(s), par, abort_flag)) goto done;
+        mbar_expect_tx(v_full(s), KV_TILE);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_load_3d(vd + c * (KV_TILE / 4), &tV, v_full(s), c * 64, j * AT_N, b * Hkv + kvh);
       }
     }
   } else if (warp == 1) {
@@ -124,10 +133,10 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t qa = smem_u32(sQ);
       auto issue_qk = [&](int j) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(kv_full(s), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(k_full(s), (j >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(s_free(s), ((j >> 1) & 1) ^ 1, abort_flag)) return false;
         fence_after();
-        const uint32_t ka = smem_u32(sKV + s * 2 * KV_TILE);
+        const uint32_t ka = smem_u32(sK + s * KV_TILE);
 #pragma unroll
         for (int ks = 0; ks < AT_D / 16; ++ks) {
           const uint32_t sub = ks >> 2, in = (ks & 3) * 32;   // 64-wide sub-tile, 16-element step
@@ -135,21 +144,23 @@ __global__ void __launch_bounds__(192, 1)
                    id_qk, ks > 0 ? 1u : 0u);
         }
         mma_commit(s_full(s));
+        mma_commit(k_empty(s));            // K slot free once these MMAs have read it
         return true;
       };
       if (n_kv > 0 && !issue_qk(0)) goto done;
       for (int j = 0; j < n_kv; ++j) {
         if (j + 1 < n_kv && !issue_qk(j + 1)) goto done;
         if (!mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag)) goto done;
+        if (!mbar_wait(v_full(j & 1), (j >> 1) & 1, abort_flag)) goto done;
         fence_after();
         const uint32_t pa = smem_u32(sP + (j & 1) * P_BYTES);
-        const uint32_t va = smem_u32(sKV + (j & 1) * 2 * KV_TILE + KV_TILE);
+        const uint32_t va = smem_u32(sV + (j & 1) * KV_TILE);
 #pragma unroll
         for (int ks = 0; ks < AT_N / 16; ++ks)
           mma_bf16(tO, sw128_desc(pa + ks * 32), sw128_desc_mn(va + ks * 2048, KV_TILE / 4), id_pv,
                    (j > 0 || ks > 0) ? 1u : 0u);
         mma_commit(pv_done(j & 1));
-        mma_commit(kv_empty(j & 1));
+        mma_commit(v_empty(j & 1));
       }
     }
   } else {
