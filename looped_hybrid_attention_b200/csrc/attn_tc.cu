@@ -5,19 +5,21 @@
 // positions (row r: head r / QT, position q0 + r % QT), so every K/V tile loaded serves
 // all heads that share it.  Warps:
 //   0     TMA: the Q tile once (per head, 4 x [QT x 64] boxes), then K and V tiles of 64
-//         keys into two separate 2-stage rings (3-D maps over the per-execution slab, so
-//         keys past Tkv read as zeros).  A K slot is free as soon as Q K^T has read it,
-//         a V slot once P V has: K tiles stream in about a tile ahead of their use
-//         instead of waiting for the previous P V;
+//         keys into two separate rings (3-D maps over the per-execution slab, so keys
+//         past Tkv read as zeros).  A K slot is free as soon as Q K^T has read it, a V
+//         slot once P V has, so K tiles stream in ahead of their use;
 //   1     MMA: S_j = Q K_j^T (M 128, N 64, K 256) into one of two TMEM buffers, and
-//         O += P_j V_j (M 128, N 256, K 64; V is an MN-major operand) into TMEM;
+//         O += P_j V_j (M 128, N 256, K 64) into TMEM, with P_j read from TMEM as the
+//         A operand and V an MN-major shared-memory operand;
 //   2..5  softmax, one thread per query row (TMEM lane = row, so the row max and
-//         sum are thread-local): scores -> exp2 -> bf16 P written to shared memory in
-//         the 128-byte-swizzled K-major layout the MMA reads; O is rescaled in TMEM
+//         sum are thread-local): scores -> exp2 -> bf16 P, packed two per column and
+//         stored over the first 32 columns of S_j's own buffer; O is rescaled in TMEM
 //         only when the running max grows by more than 2^8 (the stale max cancels in
 //         the final O / l); finally O / l * sigmoid(gate) is stored.
-// Q K^T of tile j+1 overlaps the softmax of tile j, and with two P buffers the softmax
-// of tile j+1 overlaps the P.V of tile j.  All waits are bounded.
+// Q K^T of tile j+1 overlaps the softmax of tile j.  The tensor pipe runs its MMAs in
+// issue order (Q K^T j+1, P V j, Q K^T j+2, ...), so P V j has read P_j before
+// Q K^T j+2 overwrites that buffer: no barrier is needed for the reuse.  The K ring
+// has three stages, the V ring two.  All waits are bounded.
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -27,8 +29,8 @@ namespace tc {
 constexpr int AT_M = 128, AT_N = 64, AT_D = 256;
 constexpr int Q_BYTES = AT_M * AT_D * 2;         // 64 KiB
 constexpr int KV_TILE = AT_N * AT_D * 2;         // 32 KiB each for K and V
-constexpr int P_BYTES = AT_M * AT_N * 2;         // 16 KiB
-constexpr int AT_SMEM = Q_BYTES + 2 * 2 * KV_TILE + 2 * P_BYTES + 1024 + 256;
+constexpr int K_STAGES = 3, V_STAGES = 2;
+constexpr int AT_SMEM = Q_BYTES + (K_STAGES + V_STAGES) * KV_TILE + 1024 + 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units
 
 // 2^x as one MUFU op (x <= 0 here after the row-max shift; denormal results flush to 0).
@@ -47,22 +49,20 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
   uint8_t* sK = smem + Q_BYTES;                       // K ring: stage s at s * KV_TILE
-  uint8_t* sV = sK + 2 * KV_TILE;                     // V ring
-  uint8_t* sP = sV + 2 * KV_TILE;                     // two P buffers (tile j uses j & 1)
-  uint64_t* bars = (uint64_t*)(sP + 2 * P_BYTES);
+  uint8_t* sV = sK + K_STAGES * KV_TILE;              // V ring
+  uint64_t* bars = (uint64_t*)(sV + V_STAGES * KV_TILE);
   uint32_t* tmem_slot = (uint32_t*)(bars + 17);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0;
-  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto k_empty = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (5 + s); };
-  auto v_empty = [&](int s) { return bar0 + 8u * (7 + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (9 + b); };
-  auto s_free = [&](int b) { return bar0 + 8u * (11 + b); };
-  // one p_full / pv_done per P buffer, so no barrier runs two phases ahead of its waiter
+  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };       // s < K_STAGES
+  auto k_empty = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (7 + s); };       // s < V_STAGES
+  auto v_empty = [&](int s) { return bar0 + 8u * (9 + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (11 + b); };       // b < 2
+  // one p_full / pv_done per S buffer, so no barrier runs two phases ahead of its waiter
   auto p_full = [&](int s) { return bar0 + 8u * (13 + s); };
-  auto pv_done = [&](int s) { return bar0 + 8u * (15 + s); };
+  auto pv_done = [&](int s) { return bar0 + 8u * (15 + s); };     // slots 0..16 in use
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = gridDim.x;
@@ -76,14 +76,15 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < K_STAGES; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
-      mbar_init(s_full(s), 1);
-      mbar_init(s_free(s), 128);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(s_full(s), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(p_full(s), 128);
       mbar_init(pv_done(s), 1);
@@ -112,17 +113,16 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_3d(smem_u32(sQ + c * (Q_BYTES / 4) + hh * QT * 128), &tQ, q_full, (kvh * rep + hh) * AT_D + c * 64,
                       q0, b);
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        const uint32_t par = ((j >> 1) & 1) ^ 1;
-        if (!mbar_wait(k_empty(s), par, abort_flag)) goto done;
-        mbar_expect_tx(k_full(s), KV_TILE);
-        const uint32_t kd = smem_u32(sK + s * KV_TILE), vd = smem_u32(sV + s * KV_TILE);
+        const int sk = j % K_STAGES, sv = j % V_STAGES;
+        if (!mbar_wait(k_empty(sk), ((j / K_STAGES) & 1) ^ 1, abort_flag)) goto done;
+        mbar_expect_tx(k_full(sk), KV_TILE);
+        const uint32_t kd = smem_u32(sK + sk * KV_TILE), vd = smem_u32(sV + sv * KV_TILE);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_load_3d(kd + c * (KV_TILE / 4), &tK, k_full(s), c * 64, j * AT_N, b * Hkv + kvh);
-        if (!mbar_wait(v_empty(s), par, abort_flag)) goto done;
-        mbar_expect_tx(v_full(s), KV_TILE);
+        for (int c = 0; c < 4; ++c) tma_load_3d(kd + c * (KV_TILE / 4), &tK, k_full(sk), c * 64, j * AT_N, b * Hkv + kvh);
+        if (!mbar_wait(v_empty(sv), ((j / V_STAGES) & 1) ^ 1, abort_flag)) goto done;
+        mbar_expect_tx(v_full(sv), KV_TILE);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_load_3d(vd + c * (KV_TILE / 4), &tV, v_full(s), c * 64, j * AT_N, b * Hkv + kvh);
+        for (int c = 0; c < 4; ++c) tma_load_3d(vd + c * (KV_TILE / 4), &tV, v_full(sv), c * 64, j * AT_N, b * Hkv + kvh);
       }
     }
   } else if (warp == 1) {
@@ -132,11 +132,10 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(q_full, 0, abort_flag)) goto done;
       const uint32_t qa = smem_u32(sQ);
       auto issue_qk = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(k_full(s), (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(s_free(s), ((j >> 1) & 1) ^ 1, abort_flag)) return false;
+        const int s = j & 1, sk = j % K_STAGES;
+        if (!mbar_wait(k_full(sk), (j / K_STAGES) & 1, abort_flag)) return false;
         fence_after();
-        const uint32_t ka = smem_u32(sK + s * KV_TILE);
+        const uint32_t ka = smem_u32(sK + sk * KV_TILE);
 #pragma unroll
         for (int ks = 0; ks < AT_D / 16; ++ks) {
           const uint32_t sub = ks >> 2, in = (ks & 3) * 32;   // 64-wide sub-tile, 16-element step
@@ -144,23 +143,23 @@ __global__ void __launch_bounds__(192, 1)
                    id_qk, ks > 0 ? 1u : 0u);
         }
         mma_commit(s_full(s));
-        mma_commit(k_empty(s));            // K slot free once these MMAs have read it
+        mma_commit(k_empty(sk));           // K slot free once these MMAs have read it
         return true;
       };
       if (n_kv > 0 && !issue_qk(0)) goto done;
       for (int j = 0; j < n_kv; ++j) {
         if (j + 1 < n_kv && !issue_qk(j + 1)) goto done;
+        const int sv = j % V_STAGES;
         if (!mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag)) goto done;
-        if (!mbar_wait(v_full(j & 1), (j >> 1) & 1, abort_flag)) goto done;
+        if (!mbar_wait(v_full(sv), (j / V_STAGES) & 1, abort_flag)) goto done;
         fence_after();
-        const uint32_t pa = smem_u32(sP + (j & 1) * P_BYTES);
-        const uint32_t va = smem_u32(sV + (j & 1) * KV_TILE);
+        const uint32_t pa = tmem + (uint32_t)((j & 1) * AT_N);     // P_j: bf16 pairs over 32 columns
+        const uint32_t va = smem_u32(sV + sv * KV_TILE);
 #pragma unroll
         for (int ks = 0; ks < AT_N / 16; ++ks)
-          mma_bf16(tO, sw128_desc(pa + ks * 32), sw128_desc_mn(va + ks * 2048, KV_TILE / 4), id_pv,
-                   (j > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, pa + ks * 8, sw128_desc_mn(va + ks * 2048, KV_TILE / 4), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
         mma_commit(pv_done(j & 1));
-        mma_commit(v_empty(j & 1));
+        mma_commit(v_empty(sv));
       }
     }
   } else {
@@ -180,8 +179,6 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(tmem + lane_off + s * AT_N, sa);
       tmem_ld32(tmem + lane_off + s * AT_N + 32, sb);
       tmem_wait_ld();
-      fence_before();
-      mbar_arrive(s_free(s));
       // raw scores; the max is taken before scaling (scale > 0).  Only tiles that reach
       // the causal diagonal or the end of the keys need the per-element mask.
       float t[64];
@@ -223,27 +220,21 @@ __global__ void __launch_bounds__(192, 1)
         }
         m_used = mt;
       }
-      // P buffer j & 1 was last read by the P.V of tile j - 2
-      if (j >= 2 && !mbar_wait(pv_done(j & 1), ((j >> 1) & 1) ^ 1, abort_flag)) goto done;
-      // P row (bf16) into the swizzled [128 x 64] K-major tile: 16-byte chunk c of row r
-      // sits at chunk position c ^ (r & 7)
+      // P row as bf16 pairs (key 2i in the low half of column i) over the first 32
+      // columns of this tile's S buffer, the A operand of P V
       float psum = 0.f;
-      uint8_t* prow = sP + (j & 1) * P_BYTES + r * 128;
+      uint32_t w[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(fmaf(t[c * 8 + 2 * e], scale_log2, -m_used));
-          const float p1 = ex2(fmaf(t[c * 8 + 2 * e + 1], scale_log2, -m_used));
-          psum += p0 + p1;
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2(fmaf(t[2 * i], scale_log2, -m_used));
+        const float p1 = ex2(fmaf(t[2 * i + 1], scale_log2, -m_used));
+        psum += p0 + p1;
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+        w[i] = *reinterpret_cast<const uint32_t*>(&pr);
       }
+      tmem_st32(tmem + lane_off + s * AT_N, w);
+      tmem_wait_st();
       l += psum;
-      fence_proxy_async();
       fence_before();
       mbar_arrive(p_full(j & 1));
     }
