@@ -751,6 +751,246 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
   }
 }
 
+// ------------------------------------------------------------------ tensor-core pass 1 (bf16)
+// Pass 1 for bf16 models with the chunk-local products on the tensor cores (mma.sync
+// m16n8k16, bf16 operands, fp32 accumulation).  Per (b, h, chunk), C = 64 tokens:
+//   G = inclusive cumsum of the log decays g;  KK = K K^T, QK = Q K^T        (tensor cores)
+//   A[r][s] = beta_r exp(G_r - G_s) KK[r][s]  (s < r),  P[r][s] = exp(G_r - G_s) QK[r][s]  (s <= r)
+//   T = (I + A)^-1 in fp32: the four 16 x 16 diagonal blocks by substitution, then block
+//       row i = 1..3:  T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj
+//   W = (T diag(beta gamma)) K,  U' = (T diag(beta)) V   (gamma_s = exp(G_s); tensor cores,
+//       the fp32 left factor split into two bf16 terms, hi + lo, so its rounding error is
+//       about 2^-17 instead of 2^-9)
+// W, P (bf16), U', G (fp32) go to the workspace block the tensor-core sequential pass reads.
+template <int DK, int DV>
+struct IntraTc {
+  static constexpr int C = GDN_C;
+  static constexpr int KS = DK + 8, VS = DV + 8;           // bf16 row pitches (odd multiples of 16 B)
+  static constexpr int FP = C + 4;                         // fp32 row pitch of A and T
+  static constexpr int SP = C + 8;                         // bf16 row pitch of the split factors
+  static constexpr int K_B = C * KS * 2, V_B = C * VS * 2;
+  static constexpr int SPLIT_B = 2 * C * SP * 2;           // hi + lo
+  static constexpr int QA_B = (K_B > SPLIT_B ? K_B : SPLIT_B);      // Q, later the W factors
+  static constexpr int AU_B = (C * FP * 4 > SPLIT_B ? C * FP * 4 : SPLIT_B);   // A, later the U' factors
+  static constexpr int T_B = C * FP * 4, M_B = 3 * 256 * 4, G_B = 3 * C * 4;
+  static constexpr int OFF_K = 0, OFF_V = OFF_K + K_B, OFF_QA = OFF_V + V_B, OFF_AU = OFF_QA + QA_B,
+                       OFF_T = OFF_AU + AU_B, OFF_M = OFF_T + T_B, OFF_G = OFF_M + M_B;
+  static constexpr size_t BYTES = (size_t)OFF_G + G_B;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256, 2)
+    gdn_intra_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                        const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
+                        const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int n_chunks) {
+  using L = IntraTc<DK, DV>;
+  using WLB = GdnWsB<DK, DV>;
+  constexpr int C = L::C, KS = L::KS, VS = L::VS, FP = L::FP, SP = L::SP;
+  extern __shared__ __align__(16) uint8_t smi[];
+  __nv_bfloat16* Ks = (__nv_bfloat16*)(smi + L::OFF_K);
+  __nv_bfloat16* Vs = (__nv_bfloat16*)(smi + L::OFF_V);
+  __nv_bfloat16* Qs = (__nv_bfloat16*)(smi + L::OFF_QA);
+  __nv_bfloat16* Awh = (__nv_bfloat16*)(smi + L::OFF_QA);    // after Q K^T
+  __nv_bfloat16* Awl = Awh + C * SP;
+  float* As = (float*)(smi + L::OFF_AU);
+  __nv_bfloat16* Auh = (__nv_bfloat16*)(smi + L::OFF_AU);    // after T is complete
+  __nv_bfloat16* Aul = Auh + C * SP;
+  float* Ts = (float*)(smi + L::OFF_T);
+  float* Ms = (float*)(smi + L::OFF_M);
+  float* Gs = (float*)(smi + L::OFF_G);
+  float* Bs = Gs + C;
+  float* Es = Bs + C;                                       // gamma = exp(G)
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int c0 = c * C, n = min(C, T_len - c0);
+  uint8_t* blk = ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
+  __nv_bfloat16* Pg = reinterpret_cast<__nv_bfloat16*>(blk + WLB::P_OFF);
+  __nv_bfloat16* Wg = reinterpret_cast<__nv_bfloat16*>(blk + WLB::W_OFF);
+  float* Ug = reinterpret_cast<float*>(blk + WLB::U_OFF);
+
+  // ---- 1. the chunk's K, Q, V rows (zeros past the sequence end), decays and betas
+  {
+    constexpr int RK = DK * 2 / 16, RV = DV * 2 / 16;     // 16-byte pieces per row
+    for (int idx = tid; idx < C * RK; idx += 256) {
+      const int r = idx / RK, p = idx % RK;
+      const bool ok = r < n;
+      const long row = (((long)b * T_len + c0 + (ok ? r : 0)) * H + h) * DK;
+      cp_async16(Ks + r * KS + 8 * p, k + row + 8 * p, ok);
+      cp_async16(Qs + r * KS + 8 * p, q + row + 8 * p, ok);
+    }
+    for (int idx = tid; idx < C * RV; idx += 256) {
+      const int r = idx / RV, p = idx % RV;
+      const bool ok = r < n;
+      const long row = (((long)b * T_len + c0 + (ok ? r : 0)) * H + h) * DV;
+      cp_async16(Vs + r * VS + 8 * p, v + row + 8 * p, ok);
+    }
+    cp_async_commit();
+    if (tid < C) {
+      const long gi = ((long)b * T_len + c0 + tid) * H + h;
+      Gs[tid] = tid < n ? g[gi] : 0.f;
+      Bs[tid] = tid < n ? beta[gi] : 0.f;
+    }
+    __syncthreads();
+    if (tid < 32) {                 // inclusive prefix sum of the log decays
+      const float a0 = Gs[2 * tid], a1 = a0 + Gs[2 * tid + 1];
+      float x = a1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (tid >= o) x += y;
+      }
+      Gs[2 * tid] = x - a1 + a0;
+      Gs[2 * tid + 1] = x;
+      Es[2 * tid] = expf(x - a1 + a0);
+      Es[2 * tid + 1] = expf(x);
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+  }
+  if (tid < C) reinterpret_cast<float*>(blk + WLB::G_OFF)[tid] = Gs[tid];
+
+  // ---- 2. K K^T and Q K^T on and below the diagonal; A (smem, fp32) and P (workspace, bf16)
+  {
+    const int mt = w >> 1;                                  // rows 16 mt .. 16 mt + 15
+    float akk[4][4], aqk[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) akk[i][e] = aqk[i][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < DK / 16; ++ks) {
+      uint32_t ak[4], aq[4];
+      ldsm_x4(ak, Ks + (mt * 16 + (lane & 15)) * KS + ks * 16 + (lane >> 4) * 8);
+      ldsm_x4(aq, Qs + (mt * 16 + (lane & 15)) * KS + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int nt = (w & 1) + 2 * i;                     // 8-column tiles
+        if (nt > 2 * mt + 1) break;                         // above the diagonal
+        uint32_t bk[2];
+        ldsm_x2(bk, Ks + (nt * 8 + (lane & 7)) * KS + ks * 16 + ((lane >> 3) & 1) * 8);
+        mma16816(akk[i], ak, bk);
+        mma16816(aqk[i], aq, bk);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int nt = (w & 1) + 2 * i;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = mt * 16 + gq + 8 * half, s0 = nt * 8 + 2 * tq;
+        float pv[2] = {0.f, 0.f};
+        if (nt <= 2 * mt + 1) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int s2 = s0 + e;
+            const float dec = s2 <= r ? expf(Gs[r] - Gs[s2]) : 0.f;
+            As[r * FP + s2] = s2 < r ? Bs[r] * dec * akk[i][2 * half + e] : 0.f;
+            pv[e] = dec * aqk[i][2 * half + e];
+          }
+        }
+        st_bf2(Pg + r * C + s0, pv[0], pv[1]);              // zeros above the diagonal
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. T = (I + A)^-1: diagonal 16 x 16 blocks by forward substitution (one column each)
+  if (tid < C) {
+    const int d = tid >> 4, cc = tid & 15, o = 16 * d;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = r == cc ? 1.f : 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-As[(o + r) * FP + o + s2], x[s2], acc);
+      x[r] = r < cc ? 0.f : acc;
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Ts[(o + r) * FP + o + cc] = x[r];
+  }
+  __syncthreads();
+  // block rows 1..3: M_j = sum_{k=j}^{i-1} A_ik T_kj, then T_ij = -T_ii M_j
+  for (int i = 1; i < 4; ++i) {
+    for (int e = tid; e < 256 * i; e += 256) {
+      const int j = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float acc = 0.f;
+      for (int kb = j; kb < i; ++kb)
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = fmaf(As[(16 * i + rr) * FP + 16 * kb + m], Ts[(16 * kb + m) * FP + 16 * j + cc], acc);
+      Ms[e] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 256 * i; e += 256) {
+      const int j = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m <= rr) acc = fmaf(Ts[(16 * i + rr) * FP + 16 * i + m], Ms[(j << 8) + (m << 4) + cc], acc);
+      Ts[(16 * i + rr) * FP + 16 * j + cc] = -acc;
+    }
+    __syncthreads();
+  }
+
+  // ---- 4. left factors T diag(beta gamma) and T diag(beta), each as bf16 hi + lo
+  for (int e = tid; e < C * C / 2; e += 256) {
+    const int r = e / (C / 2), s2 = 2 * (e % (C / 2));
+    float tw[2], tu[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float t = (s2 + u) <= r ? Ts[r * FP + s2 + u] : 0.f;
+      tu[u] = t * Bs[s2 + u];
+      tw[u] = tu[u] * Es[s2 + u];
+    }
+    const __nv_bfloat162 wh = __floats2bfloat162_rn(tw[0], tw[1]), uh = __floats2bfloat162_rn(tu[0], tu[1]);
+    const float2 whf = __bfloat1622float2(wh), uhf = __bfloat1622float2(uh);
+    *reinterpret_cast<__nv_bfloat162*>(Awh + r * SP + s2) = wh;
+    *reinterpret_cast<__nv_bfloat162*>(Awl + r * SP + s2) = __floats2bfloat162_rn(tw[0] - whf.x, tw[1] - whf.y);
+    *reinterpret_cast<__nv_bfloat162*>(Auh + r * SP + s2) = uh;
+    *reinterpret_cast<__nv_bfloat162*>(Aul + r * SP + s2) = __floats2bfloat162_rn(tu[0] - uhf.x, tu[1] - uhf.y);
+  }
+  __syncthreads();
+
+  // ---- 5. W = Aw K (bf16 out), U' = Au V (fp32 out): warp = (16-row tile, half of the columns)
+  {
+    const int mt = w & 3, nh = w >> 2;
+    auto product = [&](const __nv_bfloat16* Ah, const __nv_bfloat16* Al, const __nv_bfloat16* Bm, int BP, int NC,
+                       auto&& store) {
+      constexpr int NTW = (DK > DV ? DK : DV) / 16;          // 8-column tiles per warp (upper bound)
+      const int ntw = NC / 16;
+      float acc[NTW][4];
+#pragma unroll
+      for (int t2 = 0; t2 < NTW; ++t2)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t2][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks) {
+        uint32_t ah[4], al[4];
+        ldsm_x4(ah, Ah + (mt * 16 + (lane & 15)) * SP + ks * 16 + (lane >> 4) * 8);
+        ldsm_x4(al, Al + (mt * 16 + (lane & 15)) * SP + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+        for (int t2 = 0; t2 < NTW; ++t2) {
+          if (t2 >= ntw) break;
+          uint32_t bb[2];
+          ldsm_x2_t(bb, Bm + (ks * 16 + (lane & 15)) * BP + (nh * ntw + t2) * 8);
+          mma16816(acc[t2], ah, bb);
+          mma16816(acc[t2], al, bb);
+        }
+      }
+#pragma unroll
+      for (int t2 = 0; t2 < NTW; ++t2) {
+        if (t2 >= ntw) break;
+        const int col = (nh * ntw + t2) * 8 + 2 * tq, r0 = mt * 16 + gq;
+        store(r0, col, acc[t2][0], acc[t2][1]);
+        store(r0 + 8, col, acc[t2][2], acc[t2][3]);
+      }
+    };
+    product(Awh, Awl, Ks, KS, DK, [&](int r, int col, float x0, float x1) { st_bf2(Wg + r * DK + col, x0, x1); });
+    product(Auh, Aul, Vs, VS, DV, [&](int r, int col, float x0, float x1) {
+      *reinterpret_cast<float2*>(Ug + r * DV + col) = make_float2(x0, x1);
+    });
+  }
+}
+
 template <typename T, int DK, int DV>
 static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                    float* state, void* out, int B, int T_len, int H, float scale, void* workspace,
@@ -772,8 +1012,22 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k1<<<dim3(n_chunks, H, B), 256, smem1, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, (float*)workspace, T_len,
-                                               H, n_chunks);
+  if (TC) {
+    using LI = IntraTc<DK, DV>;
+    auto k1t = gdn_intra_tc_kernel<DK, DV>;
+    static bool attr_t = false;
+    if (!attr_t) {
+      cudaError_t e = cudaFuncSetAttribute(k1t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LI::BYTES);
+      if (e != cudaSuccess) return e;
+      attr_t = true;
+    }
+    k1t<<<dim3(n_chunks, H, B), 256, LI::BYTES, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                      (const __nv_bfloat16*)v, g, beta, (uint8_t*)workspace, T_len, H,
+                                                      n_chunks);
+  } else {
+    k1<<<dim3(n_chunks, H, B), 256, smem1, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, (float*)workspace,
+                                                 T_len, H, n_chunks);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (TC)
@@ -806,6 +1060,9 @@ cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* 
                       const float* beta, float* state, void* out, int B, int T, int H, int dk,
                       int dv, float scale, int dtype, cudaStream_t s, void* workspace) {
   if (T == 0 || B == 0) return cudaSuccess;
+  // the two-pass kernels copy 16-byte pieces of q, k, v rows and of the workspace
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  if (workspace && !(al16(q) && al16(k) && al16(v) && al16(workspace))) workspace = nullptr;
   if (workspace) {
     if (dk == 128 && dv == 128)
       return dtype == BF16
