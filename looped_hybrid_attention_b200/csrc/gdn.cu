@@ -597,7 +597,8 @@ struct ScanTc {
   static constexpr int W_B = C * KP * 2, Q_B = W_B, K_B = W_B, P_B = C * PP * 2, UPF_B = C * DVS * 4, G_B = C * 4;
   static constexpr int STAGE = W_B + Q_B + K_B + P_B + UPF_B + G_B;
   static constexpr int SB_B = DVS * KP * 2, UB_B = C * UP * 2;
-  static constexpr size_t BYTES = 2 * (size_t)STAGE + SB_B + 2 * UB_B;
+  static constexpr int NSTAGE = 3;                           // chunks in flight: two ahead of the one in use
+  static constexpr size_t BYTES = NSTAGE * (size_t)STAGE + SB_B + 2 * UB_B;
 };
 
 template <int DK, int DV>
@@ -611,7 +612,7 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
   constexpr int C = L::C, DVS = L::DVS, KP = L::KP, PP = L::PP, UP = L::UP;
   constexpr int NT3 = DK / 64;                               // state column tiles per warp
   extern __shared__ __align__(16) uint8_t smb[];
-  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + 2 * L::STAGE);  // [DVS][KP] bf16 copy of the state slice
+  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + L::NSTAGE * L::STAGE);  // [DVS][KP] bf16 copy of the state slice
   __nv_bfloat16* Ub = Sb + DVS * KP;                         // [C][UP] U
   __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
@@ -658,17 +659,17 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
   };
 
   issue(0, 0);
+  if (n_chunks > 1) issue(1, 1);
   const int mt = w >> 1, nt = w & 1;                         // phases 1-2: 4 x 2 output tiles
   const int r0 = mt * 16 + gq, r1 = r0 + 8, ic = nt * 8 + 2 * tq;
   for (int c = 0; c < n_chunks; ++c) {
-    const int bi = c & 1;
-    if (c + 1 < n_chunks) {
-      issue(c + 1, bi ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    const int bi = c % L::NSTAGE;
+    // chunk c's copies are done once at most one later group (chunk c + 1) is pending
+    if (c + 1 < n_chunks) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    // every warp has finished chunk c - 1, so its buffer can take chunk c + 2
     __syncthreads();
+    if (c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
     const uint8_t* base = smb + bi * L::STAGE;
     const __nv_bfloat16* Wb = (const __nv_bfloat16*)base;
     const __nv_bfloat16* Qb = (const __nv_bfloat16*)(base + L::W_B);
