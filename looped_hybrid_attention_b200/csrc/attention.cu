@@ -38,7 +38,7 @@ cudaError_t rope_table(float2* tab, int T, int pos0, int rot, float base, cudaSt
   return cudaGetLastError();
 }
 
-template <typename T, int DH>
+template <typename T, int DH, bool VEC>
 __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, int ld_p, const T* __restrict__ q_norm,
                                                       const T* __restrict__ k_norm, T* __restrict__ q_out,
                                                       T* __restrict__ k_cache, T* __restrict__ v_cache, int kv_cap,
@@ -58,15 +58,28 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
   const int kvh = hh - Hq;
   const T* src = is_q ? row + hh * DH : row + 2 * Hq * DH + kvh * DH;
   const T* gain = is_q ? q_norm : k_norm;
-  float x[PER];
+  // VEC: rows 16-byte aligned, so each lane moves its PER elements as 8-element vectors
+  constexpr bool V8 = VEC && PER % 8 == 0;
+  float x[PER], gn[PER];
+  if constexpr (V8) {
 #pragma unroll
-  for (int u = 0; u < PER; ++u) x[u] = ldf(src + lane * PER + u);
+    for (int u = 0; u < PER; u += 8) {
+      load8(src + lane * PER + u, x + u);
+      load8(gain + lane * PER + u, gn + u);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      x[u] = ldf(src + lane * PER + u);
+      gn[u] = ldf(gain + lane * PER + u);
+    }
+  }
   float ss = 0.f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) ss += x[u] * x[u];
   const float inv = rsqrtf(warp_sum(ss) / (float)DH + eps);
 #pragma unroll
-  for (int u = 0; u < PER; ++u) x[u] = x[u] * inv * ldf(gain + lane * PER + u);
+  for (int u = 0; u < PER; ++u) x[u] = x[u] * inv * gn[u];
   // rotary on dims [0, rot): pair (2j, 2j+1), angle pos * base^(-2j/rot), evaluated in fp64
 #pragma unroll
   for (int u = 0; u < PER; u += 2) {
@@ -100,11 +113,22 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
     dst = k_cache + slot;
     const T* vs = row + 2 * Hq * DH + Hkv * DH + kvh * DH;
     T* vd = v_cache + slot;
+    if constexpr (V8) {
 #pragma unroll
-    for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
+      for (int u = 0; u < PER; u += 16 / (int)sizeof(T))
+        *reinterpret_cast<uint4*>(vd + lane * PER + u) = *reinterpret_cast<const uint4*>(vs + lane * PER + u);
+    } else {
+#pragma unroll
+      for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
+    }
   }
+  if constexpr (V8) {
 #pragma unroll
-  for (int u = 0; u < PER; ++u) stf(dst + lane * PER + u, x[u]);
+    for (int u = 0; u < PER; u += 8) store8(dst + lane * PER + u, x + u);
+  } else {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) stf(dst + lane * PER + u, x[u]);
+  }
 }
 
 cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
@@ -114,8 +138,17 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
   if (T == 0 || B == 0) return cudaSuccess;
   const int warps = 8;
   dim3 grid((unsigned)(((long)T * (Hq + Hkv) + warps - 1) / warps), B);
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  const int es = dtype == BF16 ? 2 : 4;
+  const bool vec = al16(P) && al16(q_norm) && al16(k_norm) && al16(q_out) && al16(k_cache) && al16(v_cache) &&
+                   ((long)ld_p * es) % 16 == 0;
 #define FA_PREP(TT, DHV)                                                                                   \
-  fa_prep_kernel<TT, DHV><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,               \
+  do {                                                                                                     \
+    if (vec) FA_PREP_V(TT, DHV, true);                                                                     \
+    else FA_PREP_V(TT, DHV, false);                                                                        \
+  } while (0)
+#define FA_PREP_V(TT, DHV, V)                                                                              \
+  fa_prep_kernel<TT, DHV, V><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,            \
                                                       (const TT*)k_norm, (TT*)q_out, (TT*)k_cache,         \
                                                       (TT*)v_cache, kv_cap, T, pos0, Hq, Hkv, rotary_dims, \
                                                       rope_base, eps, rope_tab)
@@ -127,6 +160,7 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
     else if (dh == 64) FA_PREP(float, 64); else return cudaErrorNotSupported;
   }
 #undef FA_PREP
+#undef FA_PREP_V
   return cudaGetLastError();
 }
 

@@ -63,12 +63,56 @@ __global__ void gdn_prep_kernel(const T* __restrict__ P, int ld_p, const float* 
   }
 }
 
+// bf16, dk = dv = 128, 16-byte aligned rows: one warp per (token, head) with 16-byte
+// vectors -- lanes 0-15 normalise q, lanes 16-31 normalise k (8 elements each, sums
+// reduced within each half-warp), lanes 0-15 copy v.
+__global__ void gdn_prep_v128_kernel(const __nv_bfloat16* __restrict__ P, int ld_p, const float* __restrict__ a_bias,
+                                     const float* __restrict__ b_bias, __nv_bfloat16* __restrict__ q,
+                                     __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
+                                     float* __restrict__ g, float* __restrict__ beta, int M, int H, float eps) {
+  constexpr int D = 128;
+  const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
+  const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (w >= (long)M * H) return;
+  const long m = w / H;
+  const int h = (int)(w % H);
+  const __nv_bfloat16* row = P + m * ld_p;
+  const __nv_bfloat16* src = row + half * H * D + h * D + hl * 8;     // q (half 0) or k (half 1)
+  float x[8];
+  load8(src, x);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss + eps);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] *= inv;
+  store8((half ? k : q) + w * D + hl * 8, x);
+  if (!half)
+    *reinterpret_cast<uint4*>(v + w * D + hl * 8) = *reinterpret_cast<const uint4*>(row + 2 * H * D + h * D + hl * 8);
+  if (lane == 16) {
+    const float a = __bfloat162float(row[2 * H * D + H * D + h]) + a_bias[h];
+    const float b = __bfloat162float(row[2 * H * D + H * D + H + h]) + b_bias[h];
+    const float sp = a > 20.f ? a : log1pf(expf(a));    // softplus
+    g[w] = -sp;
+    beta[w] = 1.f / (1.f + expf(-b));
+  }
+}
+
 cudaError_t gdn_prep(const void* P, int ld_p, const float* a_bias, const float* b_bias, void* q,
                      void* k, void* v, float* g, float* beta, int M, int H, int dk, int dv,
                      float eps, int dtype, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int warps = 8;
   dim3 grid((unsigned)(((long)M * H + warps - 1) / warps));
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  if (dtype == BF16 && dk == 128 && dv == 128 && ld_p % 8 == 0 && al16(P) && al16(q) && al16(k) && al16(v)) {
+    gdn_prep_v128_kernel<<<grid, warps * 32, 0, s>>>((const __nv_bfloat16*)P, ld_p, a_bias, b_bias,
+                                                     (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, g,
+                                                     beta, M, H, eps);
+    return cudaGetLastError();
+  }
   if (dtype == BF16)
     gdn_prep_kernel<__nv_bfloat16><<<grid, warps * 32, 0, s>>>(
         (const __nv_bfloat16*)P, ld_p, a_bias, b_bias, (__nv_bfloat16*)q, (__nv_bfloat16*)k,
