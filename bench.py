@@ -198,7 +198,7 @@ def recorded_traffic(kernel):
     with open(path) as f:
         rec = json.load(f)
     src = b"".join(open(os.path.join(ROOT, "looped_hybrid_attention_b200", "csrc", n), "rb").read()
-                   for n in ("gemm_tc.cu", "tc_common.cuh"))
+                   for n in ("gemm_tc.cu", "gemm_tc2.cu", "tc_common.cuh"))
     if hashlib.sha256(src).hexdigest() != rec.get("kernel_sources_sha256"):
         return None
     return rec.get("traffic_bytes_per_launch_step_average")

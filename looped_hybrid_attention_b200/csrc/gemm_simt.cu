@@ -1,6 +1,6 @@
 // FP32-arithmetic SIMT projection Y = X W^T with fused epilogues.  This is the
 // precision path for fp32 models (tcgen05 has no fp32 MMA); bf16 projections go
-// to the tcgen05 kernel in gemm_tc.cu.  64x64 output tile, 16-deep K slices
+// to the tcgen05 kernels (gemm_tc.cu dispatch).  64x64 output tile, 16-deep K slices
 // staged transposed in shared memory, 4x4 outputs per thread.
 #include "common.cuh"
 #include "internal.h"

@@ -32,6 +32,9 @@ cudaError_t linear_skinny(const void* X, int ldx, const void* W, const void* W2,
                           void* Y, int ldy, int M, int N, int K, int epi, cudaStream_t s, void* ws,
                           size_t ws_bytes);
 size_t linear_skinny_workspace_bytes(int M, int N, int epi);
+// M > 128 (prefill): CTA pairs, 256 x 256 tiles (tcgen05 cta_group::2).
+cudaError_t linear_pair(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y,
+                        int ldy, int M, int N, int K, int epi, cudaStream_t s);
 cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, const void* R,
                         int ldr, void* Y, int ldy, int M, int N, int K, int epi, int dtype,
                         cudaStream_t s);
