@@ -275,6 +275,7 @@ __global__ void attn_rows_kernel(const T* __restrict__ q, int ld_q, const T* __r
 template <typename T, int DH>
 __global__ void attn_combine_kernel(const float* __restrict__ ws, const T* __restrict__ gate, int ld_gate,
                                     T* __restrict__ out, long rows, int Hq, int n_split) {
+  pdl_trigger();
   constexpr int PER = DH / 32;
   const int lane = threadIdx.x & 31;
   const long r = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // r = m * Hq + h
@@ -344,6 +345,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const __nv_bfloat16* _
                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ ws,
                                                           int Tkv, int q_off, int Hq, int Hkv, int causal,
                                                           int n_split, int split_len, float scale) {
+  pdl_trigger();
   using L = DecSmem<DH>;
   constexpr int PER = DH / 32;                          // dims per lane in P.V
   constexpr int CH = DH / 8;                            // 16-byte chunks per row
@@ -523,6 +525,7 @@ __global__ void __launch_bounds__(128) attn_decode_tc_kernel(const __nv_bfloat16
                                                              __nv_bfloat16* __restrict__ out, float* __restrict__ ws,
                                                              int Tkv, int q_off, int Hq, int Hkv, int causal,
                                                              int n_split, int split_len, float scale_log2) {
+  pdl_trigger();
   using L = DecTc<DH>;
   constexpr int CH = DH / 8;                                 // 16-byte chunks per K/V row
   constexpr int WD = DH / 4;                                 // head dims per warp in P.V

@@ -19,6 +19,7 @@ int read_and_clear_device_error() {
 template <typename T>
 __global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ r, T* __restrict__ sum_out,
                                const T* __restrict__ w, T* __restrict__ y, int d, long ldx, float eps) {
+  pdl_trigger();
   extern __shared__ float row[];
   __shared__ float red[32];
   const long base = (long)blockIdx.x * d;

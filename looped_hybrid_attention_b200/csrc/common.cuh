@@ -89,6 +89,12 @@ enum DeviceError : int {
 extern __device__ int g_device_error;
 __device__ __forceinline__ void set_device_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
+// Programmatic dependent launch: lets a kernel launched after this one as a programmatic
+// dependent (the few-row projections) start its prologue and weight loads now.  The
+// dependent still waits (griddepcontrol.wait) for this grid's completion before it reads
+// what this grid writes; without such a dependent this is a no-op.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 inline int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
 
 }  // namespace lk

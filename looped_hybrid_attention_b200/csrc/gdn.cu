@@ -723,21 +723,30 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
     const float* Gs = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
     const int c0 = c * C, n = min(C, T_len - c0);
     const float Glast = Gs[C - 1];
-    // phase 1 + 2a: W S^T and Q S^T share the B operand
+    // decay factors depend on G only: computed while the MMA chain below runs
+    const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
+    const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]), gl = expf(Glast);
+    // phase 1 + 2a: W S^T and Q S^T share the B operand; even and odd k-steps go to
+    // separate accumulators, halving the dependent MMA chain on the sequential path
     float cu[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
+    float cu1[4] = {0.f, 0.f, 0.f, 0.f}, cq1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < DK / 16; ++ks) {
       uint32_t aw[4], aq[4], bs[2];
       ldsm_x4(aw, Wb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
       ldsm_x4(aq, Qb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
       ldsm_x2(bs, Sb + (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8);
-      mma16816(cu, aw, bs);
-      mma16816(cq, aq, bs);
+      mma16816((ks & 1) ? cu1 : cu, aw, bs);
+      mma16816((ks & 1) ? cq1 : cq, aq, bs);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      cu[e] += cu1[e];
+      cq[e] += cq1[e];
     }
     {
       const float u00 = Upf[r0 * DVS + ic] - cu[0], u01 = Upf[r0 * DVS + ic + 1] - cu[1];
       const float u10 = Upf[r1 * DVS + ic] - cu[2], u11 = Upf[r1 * DVS + ic + 1] - cu[3];
-      const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
       st_bf2(Ub + r0 * UP + ic, u00, u01);
       st_bf2(Ub + r1 * UP + ic, u10, u11);
       st_bf2(Ueb + r0 * UP + ic, u00 * e0, u01 * e0);
@@ -754,7 +763,6 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
       mma16816(cp, ap, bu);
     }
     {
-      const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]);
       if (r0 < n)
         st_bf2(out + (((long)b * T_len + c0 + r0) * H + h) * DV + i0 + ic, scale * fmaf(g0, cq[0], cp[0]),
                scale * fmaf(g0, cq[1], cp[1]));
@@ -763,11 +771,16 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
                scale * fmaf(g1, cq[3], cp[3]));
     }
     // phase 3: S <- exp(G_last) S + Ue^T K
-    const float gl = expf(Glast);
 #pragma unroll
     for (int j = 0; j < NT3; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st[j][e] *= gl;
+    // the second half of the k-steps accumulates separately and is added at the end
+    float st1[NT3][4];
+#pragma unroll
+    for (int j = 0; j < NT3; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st1[j][e] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
       uint32_t au[4];
@@ -776,9 +789,13 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
       for (int j = 0; j < NT3; ++j) {
         uint32_t bk[2];
         ldsm_x2_t(bk, Kb + (ks * 16 + (lane & 15)) * KP + (w * NT3 + j) * 8);
-        mma16816(st[j], au, bk);
+        mma16816((ks & 1) ? st1[j] : st[j], au, bk);
       }
     }
+#pragma unroll
+    for (int j = 0; j < NT3; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[j][e] += st1[j][e];
 #pragma unroll
     for (int j = 0; j < NT3; ++j) {
       const int col = (w * NT3 + j) * 8 + 2 * tq;
@@ -1136,6 +1153,7 @@ __global__ void __launch_bounds__(256) gdn_step_kernel(const T* __restrict__ q, 
                                                        const T* __restrict__ v, const float* __restrict__ g,
                                                        const float* __restrict__ beta, float* __restrict__ state,
                                                        T* __restrict__ out, int BH, int DV, float scale) {
+  pdl_trigger();
   constexpr int PER = DK / 32;
   const int lane = threadIdx.x & 31;
   const long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
