@@ -237,6 +237,21 @@ def summarize(kernels, steps, peaks, sustained=True, tensor_bound=("gemm", "atte
     return roof, per_kernel
 
 
+def profiled(m, fn, n):
+    """Per-kernel table from the runtime's CUDA events around every launch, over n more
+    calls of fn.  Kept out of the timed regions: an event between two launches costs time
+    and stops a programmatic dependent launch from overlapping its predecessor."""
+    import torch
+    torch.cuda.synchronize()
+    m.profile(True)
+    for _ in range(n):
+        fn()
+    torch.cuda.synchronize()
+    kernels = m.profile_read()
+    m.profile(False)
+    return kernels
+
+
 def run_decode(args, m, s, dev, world, seed):
     """Decode at batch 64 over 32,768-token contexts (the decode configuration), greedy argmax.
 
@@ -251,7 +266,7 @@ def run_decode(args, m, s, dev, world, seed):
     import synth
     B, ctx = args.decode_batch, args.decode_context
     steps, warm = args.decode_steps, 3
-    c = m.cache(B, ctx + warm + 2 * steps)
+    c = m.cache(B, ctx + warm + 2 * steps + min(steps, 32))   # warm-up, timed, profiled, end to end
     stream = torch.cuda.current_stream()
     g = torch.Generator(device=dev).manual_seed(seed)
     t0 = time.time()
@@ -282,7 +297,6 @@ def run_decode(args, m, s, dev, world, seed):
         tok, nxt = nxt, tok
     torch.cuda.synchronize()
     assert L.device_error() == 0
-    m.profile(True)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -295,8 +309,8 @@ def run_decode(args, m, s, dev, world, seed):
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(ev0.elapsed_time(ev1), world)
-    kernels = m.profile_read()
-    m.profile(False)
+    prof_steps = min(steps, 32)
+    kernels = profiled(m, lambda: m.decode_step(c, tok, None, nxt, stream), prof_steps)
     # end to end: each step's token ids come from pinned host memory and the next tokens go back
     tok_host = tok.cpu().pin_memory()
     nxt_host = torch.empty_like(tok_host).pin_memory()
@@ -314,11 +328,11 @@ def run_decode(args, m, s, dev, world, seed):
     barrier(world)
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world)
     peaks = load_peaks()
-    roof, per_kernel = summarize(kernels, steps, peaks, tensor_bound=())
+    roof, per_kernel = summarize(kernels, prof_steps, peaks, tensor_bound=())
     # whole-step HBM roofline: weights per execution + KV read + GDN state read/write
     kv_bytes, st_bytes = c.nbytes()
     ctx_mid = ctx + warm + steps // 2
-    step_bytes = (sum(v["bytes"] for v in kernels.values()) / steps)
+    step_bytes = (sum(v["bytes"] for v in kernels.values()) / prof_steps)
     out = {"metric": "decode tokens/s (56-execution looped hybrid stack)", "workload":
            f"9B-shape stack, decode B={B} over {ctx}-token contexts, {steps} greedy steps",
            "value": round(B * steps * world / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms / steps, 3),
@@ -327,7 +341,8 @@ def run_decode(args, m, s, dev, world, seed):
            "setup_s": round(setup_s, 1),
            "e2e": {"value": round(B * steps * world / (ms_e2e / 1e3), 1), "unit": "tokens/s",
                    "h2d_bytes_per_step": B * 4, "d2h_bytes_per_step": B * 4},
-           "gpu_launches": sum(v["launches"] for v in kernels.values()),
+           "gpu_launches": sum(v["launches"] for v in kernels.values()) * steps // prof_steps,
+           "kernel_table_steps": prof_steps,
            "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
                              "achieved_gbs": round(step_bytes / (ms / steps / 1e3) / 1e9, 1),
                              "peak": peaks["hbm_gbs"],
@@ -356,7 +371,6 @@ def run_long(args, m, s, dev, world, seed):
     torch.cuda.synchronize()
     assert L.device_error() == 0
     assert torch.isfinite(logits).all(), "non-finite logits"
-    m.profile(True)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -369,18 +383,22 @@ def run_long(args, m, s, dev, world, seed):
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(ev0.elapsed_time(ev1), world)
-    kernels = m.profile_read()
-    m.profile(False)
+
+    def one():
+        c.reset()
+        m.prefill(c, ids, logits, stream)
+    kernels = profiled(m, one, 1)
     free, total = torch.cuda.mem_get_info(dev)
     kv_bytes, st_bytes = c.nbytes()
-    roof, per_kernel = summarize(kernels, args.long_steps, load_peaks())
+    roof, per_kernel = summarize(kernels, 1, load_peaks())
     out = {"metric": "prefill tokens/s (56-execution looped hybrid stack)",
            "workload": f"9B-shape stack, long-context prefill B=1 T={T}, bf16, random-init weights",
            "value": round(T * args.long_steps * world / (ms / 1e3), 1), "unit": "tokens/s",
            "ms_per_step": round(ms / args.long_steps, 1), "steps": args.long_steps, "warmup": 1,
            "kv_slab_bytes": kv_bytes, "gdn_state_bytes": st_bytes,
            "device_bytes_in_use": total - free,
-           "gpu_launches": sum(v["launches"] for v in kernels.values()),
+           "gpu_launches": sum(v["launches"] for v in kernels.values()) * args.long_steps,
+           "kernel_table_steps": 1,
            "roofline": roof, "kernels": per_kernel, "clocks": clk.summary()}
     del c
     return out
@@ -412,8 +430,7 @@ def run_ours(args, world, rank, local):
     assert L.device_error() == 0
     assert torch.isfinite(logits).all(), "non-finite logits"
 
-    # ---------------- device-resident timed region (with per-kernel events)
-    m.profile(True)
+    # ---------------- device-resident timed region
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -425,9 +442,8 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
     barrier(world)
     ms = ev0.elapsed_time(ev1)
-    kernels = m.profile_read()
-    m.profile(False)
     ms = max_over_ranks(ms, world)
+    kernels = profiled(m, step, 1)      # per-kernel table from one more step
     tokens = BATCH * SEQ * args.steps * world
     value = tokens / (ms / 1e3)
 
@@ -449,8 +465,8 @@ def run_ours(args, world, rank, local):
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world)
 
     peaks = load_peaks()
-    roof, per_kernel = summarize(kernels, args.steps, peaks)
-    launches = sum(v["launches"] for v in kernels.values())
+    roof, per_kernel = summarize(kernels, 1, peaks)
+    launches = sum(v["launches"] for v in kernels.values()) * args.steps
 
     line = {"metric": "prefill tokens/s (56-execution looped hybrid stack)", "value": round(value, 1),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -461,7 +477,7 @@ def run_ours(args, world, rank, local):
                        "l2": "inputs larger than L2 (16.3 GB of weights streamed per step)"},
             "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": ids.numel() * 4, "d2h_bytes_per_step": logits.numel() * 4},
-            "gpu_launches": launches, "roofline": roof, "kernels": per_kernel,
+            "gpu_launches": launches, "kernel_table_steps": 1, "roofline": roof, "kernels": per_kernel,
             "clocks": clk.summary()}
     if not args.no_decode or not args.no_long:
         del c
