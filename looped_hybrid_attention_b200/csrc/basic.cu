@@ -50,10 +50,72 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ r,
   }
 }
 
+// Register-resident variant for d = 8 * blockDim.x * CH: every thread keeps its CH
+// 8-element pieces (piece c at (c * blockDim.x + tid) * 8, so a warp's accesses are
+// contiguous) in registers across the row reduction: one read and one write per element.
+template <typename T, int CH>
+__global__ void __launch_bounds__(256) rmsnorm_reg_kernel(const T* __restrict__ x, const T* __restrict__ r,
+                                                          T* __restrict__ sum_out, const T* __restrict__ w,
+                                                          T* __restrict__ y, int d, long ldx, float eps) {
+  pdl_trigger();
+  __shared__ float red[32];
+  const long base = (long)blockIdx.x * d;
+  const long xbase = (long)blockIdx.x * ldx;
+  float a[CH][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int j = (c * blockDim.x + threadIdx.x) * 8;
+    load8(x + xbase + j, a[c]);
+    if (r) {
+      float b[8];
+      load8(r + base + j, b);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[c][i] += b[i];
+      round8<T>(a[c]);                    // the sum is what is stored and re-read downstream
+      if (sum_out) store8(sum_out + base + j, a[c]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += a[c][i] * a[c][i];
+  }
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int j = (c * blockDim.x + threadIdx.x) * 8;
+    float g[8], o[8];
+    load8(w + j, g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = a[c][i] * inv * g[i];
+    store8(y + base + j, o);
+  }
+}
+
 cudaError_t rmsnorm(const void* x, const void* r, void* sum_out, const void* w, void* y, int M,
                     int d, float eps, int dtype, cudaStream_t s, long ldx) {
   if (ldx <= 0) ldx = d;
   if (M == 0) return cudaSuccess;
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  const bool aligned = al16(x) && al16(w) && al16(y) && (!r || al16(r)) && (!sum_out || al16(sum_out)) && ldx % 8 == 0;
+  if (aligned && d % 8 == 0) {
+    const int pieces = d / 8;                    // 8-element pieces per row
+    int ch = 0, th = 0;
+    if (pieces <= 256 && pieces % 32 == 0) { ch = 1; th = pieces; }
+    else if (pieces % 256 == 0 && pieces / 256 <= 4) { ch = pieces / 256; th = 256; }
+    if (ch) {
+#define RMS_REG(TT, C) rmsnorm_reg_kernel<TT, C><<<M, th, 0, s>>>((const TT*)x, (const TT*)r, (TT*)sum_out, \
+                                                                  (const TT*)w, (TT*)y, d, ldx, eps)
+      if (dtype == BF16) {
+        if (ch == 1) RMS_REG(__nv_bfloat16, 1); else if (ch == 2) RMS_REG(__nv_bfloat16, 2);
+        else if (ch == 3) RMS_REG(__nv_bfloat16, 3); else RMS_REG(__nv_bfloat16, 4);
+      } else {
+        if (ch == 1) RMS_REG(float, 1); else if (ch == 2) RMS_REG(float, 2);
+        else if (ch == 3) RMS_REG(float, 3); else RMS_REG(float, 4);
+      }
+#undef RMS_REG
+      return cudaGetLastError();
+    }
+  }
   int threads = d >= 4096 ? 256 : 128;
   size_t smem = (size_t)d * sizeof(float);
   if (dtype == BF16)

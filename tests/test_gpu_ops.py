@@ -118,10 +118,13 @@ def test_mhc_extreme_routing_logits(cuda, N):
 
 # ----------------------------------------------------------------------------- norms, embedding, argmax
 
+@pytest.mark.parametrize("d", [4096, 256, 2048, 6144, 520])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_rmsnorm_with_residual(cuda, dtype):
+def test_rmsnorm_with_residual(cuda, dtype, d):
+    """Widths for every register layout of the row (1, 2 or 3 eight-element pieces per
+    thread) and one (d = 520) that takes the shared-memory kernel."""
     import looped_hybrid_attention_b200 as L
-    M, d = 33, 4096
+    M = 33
     x, r = rnd((M, d), 7, "x", dtype=dtype), rnd((M, d), 8, "r", dtype=dtype)
     w = rnd((d,), 9, "w", dtype=dtype, std=0.1) + 1
     y, s = torch.empty_like(x), torch.empty_like(x)
