@@ -10,9 +10,9 @@
 //   1     MMA: S_j = Q K_j^T (M 128, N 64, K 256) into one of two TMEM buffers, and
 //         O += P_j V_j (M 128, N 256, K 64) into TMEM, with P_j read from TMEM as the
 //         A operand and V an MN-major shared-memory operand;
-//   2..9  softmax in two warpgroups, two threads per query row (TMEM lane = row): each
-//         takes half of the tile's 64 keys and half of O's columns; the halves swap
-//         their row maxima through shared memory once per tile.  Scores -> exp2 ->
+//   2..9  softmax in two warpgroups, two threads per query row (TMEM lane = row): both
+//         read the tile's 64 scores for the row max, each computes P for half of the
+//         keys and rescales / writes half of O's columns.  Scores -> exp2 ->
 //         bf16 P, packed two per column and stored over the first 32 columns of S_j's
 //         own buffer; O is rescaled in TMEM only when the running max grows by more
 //         than 2^8 (the stale max cancels in the final O / l); finally
@@ -32,7 +32,7 @@ namespace tc {
 constexpr int AT_M = 128, AT_N = 64, AT_D = 256;
 constexpr int KV_TILE = AT_N * AT_D * 2;         // 32 KiB each for K and V
 constexpr int K_STAGES = 4, V_STAGES = 2;
-constexpr int XCH_BYTES = (2 * 2 + 2) * AT_M * 4;   // row-max exchange [2 tiles][2 halves][128], row sums [2][128]
+constexpr int XCH_BYTES = 2 * AT_M * 4;             // row sums of the two halves [2][128]
 constexpr int AT_SMEM = (K_STAGES + V_STAGES) * KV_TILE + 1024 + 256 + XCH_BYTES;
 constexpr int AT_THREADS = 320;                  // TMA, MMA, two softmax warpgroups
 // mbarrier slots
@@ -72,8 +72,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint8_t* sV = sK + K_STAGES * KV_TILE;              // V ring
   uint64_t* bars = (uint64_t*)(sV + V_STAGES * KV_TILE);
   uint32_t* tmem_slot = (uint32_t*)(bars + N_BARS);
-  float* xmax = (float*)((uint8_t*)bars + 256);        // [2 tiles][2 halves][AT_M]
-  float* xsum = xmax + 4 * AT_M;                       // [2 halves][AT_M]
+  float* xsum = (float*)((uint8_t*)bars + 256);        // row-sum exchange [2 halves][AT_M]
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0 + 8u * B_Q;
@@ -85,7 +84,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   // one p_full / pv_done per S buffer, so no barrier runs two phases ahead of its waiter
   auto p_full = [&](int s) { return bar0 + 8u * (B_PF + s); };
   auto pv_done = [&](int s) { return bar0 + 8u * (B_PV + s); };
-  auto x_bar = [&](int s) { return bar0 + 8u * (B_X + s); };     // row-max exchange of tile parity s
+  auto x_bar = [&](int s) { return bar0 + 8u * (B_X + s); };     // both halves done reading S (tile parity s)
   const uint32_t l_bar = bar0 + 8u * B_L;                         // row-sum exchange
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -184,9 +183,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     // ------------------------------------------------------------------ softmax: two warpgroups
     // Warps 2-5 and 6-9 reach the same TMEM lanes (lane quarter = warp % 4), so every
     // row has two threads: `half` 0 takes keys 0-31 of each tile and O columns 0-127,
-    // half 1 keys 32-63 and O columns 128-255.  The two exchange their tile maximum
-    // through shared memory (double-buffered, one mbarrier round per tile), so both make
-    // the same lazy-rescale decision; each writes its 16 columns of P.
+    // half 1 keys 32-63 and O columns 128-255.  Both read all 64 scores, so they take
+    // the same lazy-rescale decision without a hand-off; each writes its 16 columns of
+    // P once both have finished reading S (one mbarrier round per tile).
     const int quarter = warp & 3, half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                // MMA row: head r / QT, query q0 + r % QT
     const int qi = r % QT;
@@ -217,35 +216,36 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const int s = j & 1;
       if (!mbar_wait(s_full(s), (j >> 1) & 1, abort_flag)) goto done;
       fence_after();
-      uint32_t sa[32];
-      tmem_ld32(tmem + lane_off + s * AT_N + half * 32, sa);
+      // both threads of a row read all 64 scores (the row max needs them all; reading
+      // twice from TMEM is cheaper than a hand-off between the two threads)
+      uint32_t sa[32], sb[32];
+      tmem_ld32(tmem + lane_off + s * AT_N + half * 32, sa);          // this half's keys
+      tmem_ld32(tmem + lane_off + s * AT_N + (half ^ 1) * 32, sb);    // the other half's
       tmem_wait_ld();
       // raw scores; the max is taken before scaling (scale > 0).  Only tiles that reach
       // the causal diagonal or the end of the keys need the per-element mask.
       float t[32];
       float mh = -INFINITY;
-      const int kbase = j * AT_N + half * 32;
+      const int kbase = j * AT_N + half * 32, kother = j * AT_N + (half ^ 1) * 32;
       const bool all_visible = j * AT_N + AT_N <= Tkv && (!causal || j * AT_N + AT_N - 1 <= q_off + q0);
       if (all_visible) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           t[i] = __uint_as_float(sa[i]);
-          mh = fmaxf(mh, t[i]);
+          mh = fmaxf(mh, fmaxf(t[i], __uint_as_float(sb[i])));
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int key = kbase + i;
+          const int key = kbase + i, key2 = kother + i;
           const bool ok = key < Tkv && (!causal || key <= qpos);
+          const bool ok2 = key2 < Tkv && (!causal || key2 <= qpos);
           t[i] = ok ? __uint_as_float(sa[i]) : -INFINITY;
-          mh = fmaxf(mh, t[i]);
+          mh = fmaxf(mh, fmaxf(t[i], ok2 ? __uint_as_float(sb[i]) : -INFINITY));
         }
       }
-      // the row maximum over both halves (every processed tile has a visible key per row)
-      xmax[(s * 2 + half) * AT_M + r] = mh;
-      mbar_arrive(x_bar(s));
-      if (!mbar_wait(x_bar(s), (j >> 1) & 1, abort_flag)) goto done;
-      const float mt = fmaxf(mh, xmax[(s * 2 + (half ^ 1)) * AT_M + r]) * scale_log2;
+      // the row maximum of the tile (every processed tile has a visible key per row)
+      const float mt = mh * scale_log2;
       if (mt > m_used + RESCALE_THRESHOLD) {
         if (j > 0) {                                  // O holds tiles < j scaled by 2^-m_used
           if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) goto done;
@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
         w[i] = *reinterpret_cast<const uint32_t*>(&pr);
       }
+      // the partner may still be reading S columns 16-31 (which P overwrites): both
+      // threads pass this barrier after their S loads have completed
+      mbar_arrive(x_bar(s));
+      if (!mbar_wait(x_bar(s), (j >> 1) & 1, abort_flag)) goto done;
       tmem_st16(tmem + lane_off + s * AT_N + half * 16, w);
       tmem_wait_st();
       l += psum;
