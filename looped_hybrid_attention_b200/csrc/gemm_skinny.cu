@@ -29,17 +29,20 @@ namespace sk {
 
 constexpr int BW = 128;     // weight rows per tile (MMA M)
 constexpr int BK = 64;      // K per stage (one 128-byte swizzle row of bf16)
-constexpr int MIN_KB = 4;   // fewest k-blocks a CTA is given (fewer only adds partial sums)
+constexpr int MIN_KB = 8;   // fewest k-blocks a CTA is given (fewer only adds partial sums)
 
 template <int NB, int NMAT>
 struct Cfg {
   static constexpr int A_BYTES = BW * BK * 2;                     // one weight matrix
   static constexpr int B_BYTES = NB * BK * 2;                     // the activations
   static constexpr int STAGE_BYTES = NMAT * A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (200 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 10 ? 10 : STAGES_FIT;
   static constexpr int ACC_COLS = NMAT * NB;                      // one accumulator
   static constexpr int TMEM_COLS = 2 * ACC_COLS;                  // double-buffered (power of two >= 32)
+  // two CTAs per SM when their accumulators fit TMEM together: one CTA's ramp and
+  // split-tile tail then overlap the other's streaming
+  static constexpr int PER_SM = TMEM_COLS <= 256 ? 2 : 1;
+  static constexpr int STAGES_FIT = (200 * 1024 / PER_SM) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 10 ? 10 : STAGES_FIT;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
   static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation");
@@ -89,7 +92,7 @@ __device__ __forceinline__ void put_chunk(void* Y, int ldy, const __nv_bfloat16*
 }
 
 template <int NB, int NMAT, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, Cfg<NB, NMAT>::PER_SM)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tW, const __grid_constant__ CUtensorMap tW2,
                        const __grid_constant__ CUtensorMap tX, void* __restrict__ Y, int ldy,
                        const __nv_bfloat16* R, int ldr, int M, int N, int K, int whole_tiles,
@@ -373,7 +376,7 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
     grid = n_tiles;
     whole_tiles = 1;
   }
-  if (grid > num_sms()) grid = num_sms();
+  if (grid > (long)C::PER_SM * num_sms()) grid = (long)C::PER_SM * num_sms();
   int* cnt = split ? (int*)ws : nullptr;
   float* acc = split ? (float*)((char*)ws + (ws_bytes_for(M, N, EPI) - (size_t)NMAT * ((M + 3) & ~3) * N * 4))
                      : nullptr;
