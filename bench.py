@@ -157,13 +157,20 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest of every rank's x (device time is taken as the max over ranks)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, ms):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
 
 
 def run_reference(args, world, rank):
@@ -445,7 +452,7 @@ def run_ours(args, world, rank, local):
     ms = max_over_ranks(ms, world)
     kernels = profiled(m, step, 1)      # per-kernel table from one more step
     tokens = BATCH * SEQ * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = weak_scaling_value(BATCH * SEQ * args.steps, world, ms)
 
     # ---------------- end to end through the public API with host buffers
     ids_host = ids.cpu().pin_memory()
