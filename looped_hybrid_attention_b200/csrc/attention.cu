@@ -462,12 +462,10 @@ static cudaError_t launch_decode(const void* q, int ld_q, const void* k, const v
   using L = DecSmem<DH>;
   const int n_split = workspace ? attn_splits(B, 1, Tkv, Hkv) : 1;
   const int split_len = (((Tkv + n_split - 1) / n_split) + DEC_KT - 1) / DEC_KT * DEC_KT;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  {
+    cudaError_t e = set_smem_limit(attn_decode_kernel<DH>,
                                          (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid(n_split, Hkv, B);
   attn_decode_kernel<DH><<<grid, 128, L::BYTES, s>>>(
@@ -691,12 +689,10 @@ static cudaError_t launch_decode_tc(const void* q, int ld_q, const void* k, cons
   using L = DecTc<DH>;
   const int n_split = workspace ? attn_splits(B, 1, Tkv, Hkv) : 1;
   const int split_len = (((Tkv + n_split - 1) / n_split) + DTC_KT - 1) / DTC_KT * DTC_KT;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  {
+    cudaError_t e = set_smem_limit(attn_decode_tc_kernel<DH>,
                                          (int)L::BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid(n_split, Hkv, B);
   attn_decode_tc_kernel<DH><<<grid, 128, L::BYTES, s>>>(

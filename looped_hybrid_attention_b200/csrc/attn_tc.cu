@@ -350,11 +350,9 @@ cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, i
   CUtensorMap mK, mV;
   if (!make_map_3d(&mK, k, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
   if (!make_map_3d(&mV, v, AT_D, Tkv, (long)B * Hkv, AT_D, (long)kv_cap * AT_D, 64, AT_N)) return cudaErrorNotSupported;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+  {
+    cudaError_t e = set_smem_limit(attn_tc_kernel, AT_SMEM);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid((Tq + QT - 1) / QT, Hkv, B);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)AT_D);

@@ -4,6 +4,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 namespace lk {
 
 // ------------------------------------------------------------------ storage types
@@ -96,5 +100,23 @@ __device__ __forceinline__ void set_device_error(int code) { atomicCAS(&g_device
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 inline int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+// ------------------------------------------------------------------ host: launch set-up
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device): the attribute
+// belongs to the current device, so a process that drives several GPUs sets it on each.
+template <typename K>
+inline cudaError_t set_smem_limit(K kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
+}
 
 }  // namespace lk

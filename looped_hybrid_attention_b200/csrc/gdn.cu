@@ -1066,22 +1066,18 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
   auto k2t = gdn_scan_tc_kernel<DK, DV>;
   using L = ScanSmem<T, DK, DV, DVS>;
   using LT = ScanTc<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k2t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LT::BYTES);
+  {
+    cudaError_t e = set_smem_limit(k1, (int)smem1);
+    if (e == cudaSuccess) e = set_smem_limit(k2, (int)L::BYTES);
+    if (e == cudaSuccess) e = set_smem_limit(k2t, (int)LT::BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   if (TC) {
     using LI = IntraTc<DK, DV>;
     auto k1t = gdn_intra_tc_kernel<DK, DV>;
-    static bool attr_t = false;
-    if (!attr_t) {
-      cudaError_t e = cudaFuncSetAttribute(k1t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LI::BYTES);
+    {
+      cudaError_t e = set_smem_limit(k1t, (int)LI::BYTES);
       if (e != cudaSuccess) return e;
-      attr_t = true;
     }
     k1t<<<dim3(n_chunks, H, B), 256, LI::BYTES, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                                       (const __nv_bfloat16*)v, g, beta, (uint8_t*)workspace, T_len, H,
@@ -1110,7 +1106,7 @@ static cudaError_t launch_chunk(const void* q, const void* k, const void* v, con
                                 int dv, float scale, cudaStream_t s) {
   using L = GdnSmem<DK, DVS>;
   auto kern = gdn_chunk_kernel<T, DK, DVS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+  cudaError_t e = set_smem_limit(kern, (int)L::bytes);
   if (e != cudaSuccess) return e;
   dim3 grid(dv / DVS, H, B);
   kern<<<grid, 256, L::bytes, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out, T_len, H,

@@ -360,11 +360,9 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
   }
   if (!make_map(&tX, X, M, K, ldx, NB)) return cudaErrorNotSupported;
   auto kern = gemm_skinny_kernel<NB, NMAT, EPI>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  {
+    cudaError_t e = set_smem_limit(kern, (int)C::SMEM);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const long n_tiles = (N + BW - 1) / BW, kb_n = (K + BK - 1) / BK;
   const bool split = ws != nullptr && ((uintptr_t)ws % 16) == 0 && ws_bytes >= ws_bytes_for(M, N, EPI);

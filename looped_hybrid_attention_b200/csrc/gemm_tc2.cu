@@ -286,11 +286,9 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
     tB2 = tB;
   }
   auto kern = gemm_pair_kernel<EPI>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+  {
+    cudaError_t e = set_smem_limit(kern, (int)SMEM);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const long tiles = (long)((M + 2 * BM - 1) / (2 * BM)) * ((N + OUT_COLS - 1) / OUT_COLS);
   const long pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;

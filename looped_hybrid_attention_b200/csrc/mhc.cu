@@ -683,7 +683,7 @@ static cudaError_t launch_cluster(const void* X_in, const void* F, const float* 
                                   float eps, int iters, cudaStream_t s) {
   auto kern = mhc_cluster_kernel<TB, NCH, MODE>;
   const size_t bytes = MhcCl<TB, NCH>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  cudaError_t e = set_smem_limit(kern, (int)bytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(((long)N + TB - 1) / TB * CL));

@@ -168,14 +168,18 @@ inline bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long
   return r == CUDA_SUCCESS;
 }
 
+// SM count of the current device (cached per device).
 inline int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!n[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 1;
   }
-  return n;
+  return n[dev];
 }
 
 
