@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mma_sync.cuh"
+#include "tc_common.cuh"
 
 namespace lk {
 
@@ -635,31 +636,59 @@ __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float x, float y) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
 }
 
+// Shared-memory plan of the tensor-core scan.  A chunk's W, Q, K (64 x dk bf16) and P
+// (64 x 64 bf16) arrive by TMA as 64-column halves of [64 rows x 128 B] with the 128-byte
+// swizzle (16-byte chunk j of row r stored at j ^ (r & 7)); U' (this CTA's 16 columns,
+// fp32) and G (fp32) as plain boxes.  Nine tile loads per chunk, completing on the
+// stage's mbarrier.
 template <int DK, int DV>
 struct ScanTc {
-  static constexpr int C = GDN_C, DVS = 16, KP = DK + 8, PP = C + 8, UP = DVS + 8;
-  static constexpr int W_B = C * KP * 2, Q_B = W_B, K_B = W_B, P_B = C * PP * 2, UPF_B = C * DVS * 4, G_B = C * 4;
-  static constexpr int STAGE = W_B + Q_B + K_B + P_B + UPF_B + G_B;
+  static constexpr int C = GDN_C, DVS = 16, KP = DK + 8, UP = DVS + 8;
+  static constexpr int HALF = C * 128;                       // one 64-column half, 8 KB
+  static constexpr int W_B = (DK / 64) * HALF, Q_B = W_B, K_B = W_B, P_B = HALF, UPF_B = C * DVS * 4, G_B = C * 4;
+  static constexpr int TX = W_B + Q_B + K_B + P_B + UPF_B + G_B;     // bytes per chunk
+  static constexpr int STAGE = (TX + 1023) / 1024 * 1024;            // swizzled tiles: 1024-byte aligned
   static constexpr int SB_B = DVS * KP * 2, UB_B = C * UP * 2;
   static constexpr int NSTAGE = 3;                           // chunks in flight: two ahead of the one in use
-  static constexpr size_t BYTES = NSTAGE * (size_t)STAGE + SB_B + 2 * UB_B;
+  static constexpr int BAR_OFF = NSTAGE * STAGE + SB_B + 2 * UB_B;   // NSTAGE mbarriers, then an abort flag
+  static constexpr size_t BYTES = (size_t)BAR_OFF + 8 * NSTAGE + 16 + 1024;   // + alignment slack
+  static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
 };
 
+// Byte offset of bf16 element (row, col) (col a multiple of 8) in a tile stored as 64-column
+// halves of [GDN_C rows x 128 B] with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_off(int row, int col) {
+  return (uint32_t)((col >> 6) * (GDN_C * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* __restrict__ q,
-                                                          const __nv_bfloat16* __restrict__ k,
-                                                          const uint8_t* __restrict__ ws, float* __restrict__ state,
+__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap mW,
+                                                          const __grid_constant__ CUtensorMap mP,
+                                                          const __grid_constant__ CUtensorMap mU,
+                                                          const __grid_constant__ CUtensorMap mG,
+                                                          const __grid_constant__ CUtensorMap mQ,
+                                                          const __grid_constant__ CUtensorMap mK, float* __restrict__ state,
                                                           __nv_bfloat16* __restrict__ out, int T_len, int H,
                                                           int n_chunks, float scale) {
   using L = ScanTc<DK, DV>;
-  using WLB = GdnWsB<DK, DV>;
-  constexpr int C = L::C, DVS = L::DVS, KP = L::KP, PP = L::PP, UP = L::UP;
+  constexpr int C = L::C, DVS = L::DVS, KP = L::KP, UP = L::UP;
   constexpr int NT3 = DK / 64;                               // state column tiles per warp
-  extern __shared__ __align__(16) uint8_t smb[];
+  extern __shared__ __align__(16) uint8_t smb_raw[];
+  uint8_t* smb = (uint8_t*)(((uintptr_t)smb_raw + 1023) & ~(uintptr_t)1023);
   __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + L::NSTAGE * L::STAGE);  // [DVS][KP] bf16 copy of the state slice
   __nv_bfloat16* Ub = Sb + DVS * KP;                         // [C][UP] U
   __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U
+  uint64_t* full = reinterpret_cast<uint64_t*>(smb + L::BAR_OFF);   // a chunk's tiles landed, per stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + L::NSTAGE);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  if (tid == 0) {
+    for (int i = 0; i < L::NSTAGE; ++i) tc::mbar_init(tc::smem_u32(full + i), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mW) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mQ) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mK) : "memory");
+  }
   const int i0 = blockIdx.x * DVS, h = blockIdx.y, b = blockIdx.z;
   float* Sg = state + (((long)b * H + h) * DV + i0) * DK;
 
@@ -675,50 +704,43 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
     st_bf2(Sb + (gq + 8) * KP + col, st[j][2], st[j][3]);
   }
 
+  // one thread: the chunk's nine tiles (rows past the sequence end read as zeros)
   auto issue = [&](int c, int bi) {
     uint8_t* base = smb + bi * L::STAGE;
-    const uint8_t* blk = ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
-    const int c0 = c * C, n = min(C, T_len - c0);
-    constexpr int RP = DK * 2 / 16;                          // 16-byte pieces per row
-    for (int idx = tid; idx < C * RP; idx += 256) {
-      const int r = idx / RP, p = idx % RP;
-      cp_async16(base + r * KP * 2 + 16 * p, blk + WLB::W_OFF + r * DK * 2 + 16 * p, true);
-      const bool ok = r < n;
-      const long row = (((long)b * T_len + c0 + (ok ? r : 0)) * H + h) * DK;
-      cp_async16(base + L::W_B + r * KP * 2 + 16 * p, (const uint8_t*)(q + row) + 16 * p, ok);
-      cp_async16(base + L::W_B + L::Q_B + r * KP * 2 + 16 * p, (const uint8_t*)(k + row) + 16 * p, ok);
+    const int blk = ((b * H + h) * n_chunks + c);
+    const uint32_t fb = tc::smem_u32(full + bi);
+    tc::fence_proxy_async();                                 // earlier generic reads of this stage first
+    tc::mbar_expect_tx(fb, (uint32_t)L::TX);
+#pragma unroll
+    for (int hf = 0; hf < DK / 64; ++hf) {
+      tc::tma_load_3d(tc::smem_u32(base + hf * L::HALF), &mW, fb, hf * 64, 0, blk);
+      tc::tma_load_4d(tc::smem_u32(base + L::W_B + hf * L::HALF), &mQ, fb, hf * 64, h, c * C, b);
+      tc::tma_load_4d(tc::smem_u32(base + L::W_B + L::Q_B + hf * L::HALF), &mK, fb, hf * 64, h, c * C, b);
     }
-    for (int idx = tid; idx < C * (C * 2 / 16); idx += 256) {
-      const int r = idx / (C * 2 / 16), p = idx % (C * 2 / 16);
-      cp_async16(base + L::W_B + L::Q_B + L::K_B + r * PP * 2 + 16 * p, blk + WLB::P_OFF + r * C * 2 + 16 * p, true);
-    }
-    for (int idx = tid; idx < C * DVS / 4; idx += 256) {
-      const int r = idx / (DVS / 4), p = idx % (DVS / 4);
-      cp_async16(base + L::W_B + L::Q_B + L::K_B + L::P_B + r * DVS * 4 + 16 * p,
-                 blk + WLB::U_OFF + (r * DV + i0) * 4 + 16 * p, true);
-    }
-    if (tid < C / 4)
-      cp_async16(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B + 16 * tid, blk + WLB::G_OFF + 16 * tid, true);
-    cp_async_commit();
+    const int off_p = L::W_B + L::Q_B + L::K_B;
+    tc::tma_load_3d(tc::smem_u32(base + off_p), &mP, fb, 0, 0, blk);
+    tc::tma_load_3d(tc::smem_u32(base + off_p + L::P_B), &mU, fb, i0, 0, blk);
+    tc::tma_load_2d(tc::smem_u32(base + off_p + L::P_B + L::UPF_B), &mG, fb, 0, blk);
   };
 
-  issue(0, 0);
-  if (n_chunks > 1) issue(1, 1);
+  __syncthreads();                                           // barriers initialised
+  if (tid == 0) {
+    issue(0, 0);
+    if (n_chunks > 1) issue(1, 1);
+  }
   const int mt = w >> 1, nt = w & 1;                         // phases 1-2: 4 x 2 output tiles
   const int r0 = mt * 16 + gq, r1 = r0 + 8, ic = nt * 8 + 2 * tq;
   for (int c = 0; c < n_chunks; ++c) {
     const int bi = c % L::NSTAGE;
-    // chunk c's copies are done once at most one later group (chunk c + 1) is pending
-    if (c + 1 < n_chunks) cp_async_wait<1>();
-    else cp_async_wait<0>();
+    if (!tc::mbar_wait(tc::smem_u32(full + bi), (uint32_t)((c / L::NSTAGE) & 1), abort_flag)) break;
     // every warp has finished chunk c - 1, so its buffer can take chunk c + 2
     __syncthreads();
-    if (c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
+    if (tid == 0 && c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
     const uint8_t* base = smb + bi * L::STAGE;
-    const __nv_bfloat16* Wb = (const __nv_bfloat16*)base;
-    const __nv_bfloat16* Qb = (const __nv_bfloat16*)(base + L::W_B);
-    const __nv_bfloat16* Kb = (const __nv_bfloat16*)(base + L::W_B + L::Q_B);
-    const __nv_bfloat16* Pb = (const __nv_bfloat16*)(base + L::W_B + L::Q_B + L::K_B);
+    const uint8_t* Wb = base;                                // swizzled tiles (sw_off)
+    const uint8_t* Qb = base + L::W_B;
+    const uint8_t* Kb = base + L::W_B + L::Q_B;
+    const uint8_t* Pb = base + L::W_B + L::Q_B + L::K_B;
     const float* Upf = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B);
     const float* Gs = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
     const int c0 = c * C, n = min(C, T_len - c0);
@@ -733,8 +755,8 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
 #pragma unroll
     for (int ks = 0; ks < DK / 16; ++ks) {
       uint32_t aw[4], aq[4], bs[2];
-      ldsm_x4(aw, Wb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
-      ldsm_x4(aq, Qb + (mt * 16 + (lane & 15)) * KP + ks * 16 + (lane >> 4) * 8);
+      ldsm_x4(aw, Wb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
+      ldsm_x4(aq, Qb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
       ldsm_x2(bs, Sb + (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8);
       mma16816((ks & 1) ? cu1 : cu, aw, bs);
       mma16816((ks & 1) ? cq1 : cq, aq, bs);
@@ -758,7 +780,7 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
       uint32_t ap[4], bu[2];
-      ldsm_x4(ap, Pb + (mt * 16 + (lane & 15)) * PP + ks * 16 + (lane >> 4) * 8);
+      ldsm_x4(ap, Pb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
       ldsm_x2_t(bu, Ub + (ks * 16 + (lane & 15)) * UP + nt * 8);
       mma16816(cp, ap, bu);
     }
@@ -788,7 +810,7 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __nv_bfloat16* _
 #pragma unroll
       for (int j = 0; j < NT3; ++j) {
         uint32_t bk[2];
-        ldsm_x2_t(bk, Kb + (ks * 16 + (lane & 15)) * KP + (w * NT3 + j) * 8);
+        ldsm_x2_t(bk, Kb + sw_off(ks * 16 + (lane & 15), (w * NT3 + j) * 8));
         mma16816((ks & 1) ? st1[j] : st[j], au, bk);
       }
     }
@@ -1088,11 +1110,29 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (TC)
-    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                          (const uint8_t*)workspace, state, (__nv_bfloat16*)out, T_len,
-                                                          H, n_chunks, scale);
-  else
+  if (TC) {
+    // tensor maps of the workspace blocks and of q, k [B, T, H, dk] for the scan's tile loads
+    using WLB = GdnWsB<DK, DV>;
+    const uint8_t* wsb = (const uint8_t*)workspace;
+    const cuuint64_t nblk = (cuuint64_t)B * H * n_chunks, bs = (cuuint64_t)WLB::BYTES;
+    CUtensorMap mW, mP, mU, mG, mQ, mK;
+    const cuuint64_t dW[3] = {DK, GDN_C, nblk}, sW[2] = {DK * 2, bs};
+    const cuuint64_t dP[3] = {GDN_C, GDN_C, nblk}, sP[2] = {GDN_C * 2, bs};
+    const cuuint64_t dU[3] = {DV, GDN_C, nblk}, sU[2] = {DV * 4, bs};
+    const cuuint64_t dG[2] = {GDN_C, nblk}, sG[1] = {bs};
+    const cuuint64_t dQ[4] = {DK, (cuuint64_t)H, (cuuint64_t)T_len, (cuuint64_t)B};
+    const cuuint64_t sQ[3] = {DK * 2, (cuuint64_t)H * DK * 2, (cuuint64_t)T_len * H * DK * 2};
+    const cuuint32_t b64[3] = {64, GDN_C, 1}, bU[3] = {LT::DVS, GDN_C, 1}, bG[2] = {GDN_C, 1}, bQ[4] = {64, 1, GDN_C, 1};
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (!tc::make_map_nd(&mW, BF, 3, wsb + WLB::W_OFF, dW, sW, b64, true) ||
+        !tc::make_map_nd(&mP, BF, 3, wsb + WLB::P_OFF, dP, sP, b64, true) ||
+        !tc::make_map_nd(&mU, F32, 3, wsb + WLB::U_OFF, dU, sU, bU, false) ||
+        !tc::make_map_nd(&mG, F32, 2, wsb + WLB::G_OFF, dG, sG, bG, false) ||
+        !tc::make_map_nd(&mQ, BF, 4, q, dQ, sQ, bQ, true) || !tc::make_map_nd(&mK, BF, 4, k, dQ, sQ, bQ, true))
+      return cudaErrorNotSupported;
+    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>(mW, mP, mU, mG, mQ, mK, state, (__nv_bfloat16*)out, T_len, H,
+                                                          n_chunks, scale);
+  } else
     k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,
                                                     T_len, H, n_chunks, scale);
   return cudaGetLastError();
