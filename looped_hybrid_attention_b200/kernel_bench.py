@@ -45,6 +45,7 @@ def main():
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--no-ws", action="store_true", help="gemm: no partial-sum workspace (whole tiles per CTA)")
     a = ap.parse_args()
     dev = torch.device("cuda")
     g = torch.Generator(device=dev).manual_seed(0)
@@ -59,7 +60,7 @@ def main():
         epi = {"store": L.EPI_STORE, "add": L.EPI_ADD, "swiglu": L.EPI_SWIGLU, "f32": L.EPI_F32}[a.epi]
         # zero-filled partial-sum workspace for few rows (M <= 128), as the runtime gives it
         nws = L.linear_workspace_bytes(a.M, a.N, a.K, epi)
-        ws = torch.zeros(nws // 4 + 1, device=dev) if nws else None
+        ws = torch.zeros(nws // 4 + 1, device=dev) if nws and not a.no_ws else None
         ms = timed(lambda: L.linear(X, W, Y, epi, W2=W2, R=R, workspace=ws), a.warmup, a.iters)
         nmat = 2 if a.epi == "swiglu" else 1
         flops = 2.0 * a.M * a.N * a.K * nmat
