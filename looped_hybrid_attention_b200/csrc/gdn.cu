@@ -1182,9 +1182,34 @@ cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* 
 }
 
 // ------------------------------------------------------------------ single-token step
-// One warp per state row (b, h, i): the row streams through registers once
-// (read 4*dk bytes, write 4*dk bytes), two warp reductions.
-template <typename T, int DK>
+// One warp per R state rows (b, h, i0 .. i0 + R - 1) of one head: every row streams
+// through registers once (read 4*dk bytes, write 4*dk bytes, 16-byte accesses), all R
+// rows' loads are in flight together, and the head's k and q are read once for them.
+// VEC: 16-byte (dk 128) or 8-byte (dk 64) state accesses, for an aligned state.
+template <int PER>
+struct Vec;
+template <>
+struct Vec<4> {
+  static __device__ __forceinline__ void ld(const float* p, float* x) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  }
+  static __device__ __forceinline__ void st(float* p, const float* x) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+};
+template <>
+struct Vec<2> {
+  static __device__ __forceinline__ void ld(const float* p, float* x) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  }
+  static __device__ __forceinline__ void st(float* p, const float* x) {
+    *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+  }
+};
+
+template <typename T, int DK, int R, bool VEC>
 __global__ void __launch_bounds__(256) gdn_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                        const T* __restrict__ v, const float* __restrict__ g,
                                                        const float* __restrict__ beta, float* __restrict__ state,
@@ -1192,33 +1217,49 @@ __global__ void __launch_bounds__(256) gdn_step_kernel(const T* __restrict__ q, 
   pdl_trigger();
   constexpr int PER = DK / 32;
   const int lane = threadIdx.x & 31;
-  const long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= (long)BH * DV) return;
-  const long bh = row / DV;
-  const int i = (int)(row % DV);
-  float* S = state + row * DK;
-  float s[PER], kk[PER], qq[PER];
+  const long row0 = ((long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * R;
+  if (row0 >= (long)BH * DV) return;
+  const long bh = row0 / DV;                     // DV % R == 0: the R rows share the head
+  const int i0 = (int)(row0 % DV);
+  float* S = state + row0 * DK + lane * PER;
+  float s[R][PER], kk[PER], qq[PER];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (VEC) {
+      Vec<PER>::ld(S + r * DK, s[r]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < PER; ++u) s[r][u] = S[r * DK + u];
+    }
+  }
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    s[u] = S[lane * PER + u];
     kk[u] = ldf(k + bh * DK + lane * PER + u);
     qq[u] = ldf(q + bh * DK + lane * PER + u);
   }
   const float alpha = expf(g[bh]), bt = beta[bh];
-  float pred = 0.f;
 #pragma unroll
-  for (int u = 0; u < PER; ++u) pred = fmaf(s[u], kk[u], pred);
-  pred = warp_sum(pred) * alpha;
-  const float uu = bt * (ldf(v + bh * DV + i) - pred);
-  float o = 0.f;
+  for (int r = 0; r < R; ++r) {
+    float pred = 0.f;
 #pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    s[u] = fmaf(alpha, s[u], uu * kk[u]);
-    o = fmaf(s[u], qq[u], o);
-    S[lane * PER + u] = s[u];
+    for (int u = 0; u < PER; ++u) pred = fmaf(s[r][u], kk[u], pred);
+    pred = warp_sum(pred) * alpha;
+    const float uu = bt * (ldf(v + bh * DV + i0 + r) - pred);
+    float o = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      s[r][u] = fmaf(alpha, s[r][u], uu * kk[u]);
+      o = fmaf(s[r][u], qq[u], o);
+    }
+    if (VEC) {
+      Vec<PER>::st(S + r * DK, s[r]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < PER; ++u) S[r * DK + u] = s[r][u];
+    }
+    o = warp_sum(o);
+    if (lane == 0) stf(out + bh * DV + i0 + r, scale * o);
   }
-  o = warp_sum(o);
-  if (lane == 0) stf(out + bh * DV + i, scale * o);
 }
 
 cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -1226,26 +1267,28 @@ cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g
                      cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   const long rows = (long)B * H * dv;
-  dim3 grid((unsigned)((rows + 7) / 8));
+  // four rows of one head per warp, 16/8-byte state accesses; else the plain form
+  const bool r4 = dv % 4 == 0 && (uintptr_t)state % (dk == 128 ? 16 : 8) == 0;
+  const dim3 grid((unsigned)((rows + (r4 ? 31 : 7)) / (r4 ? 32 : 8)));
+#define GDN_STEP(TT, DKK, RR)                                                                                      \
+  gdn_step_kernel<TT, DKK, RR, (RR > 1)><<<grid, 256, 0, s>>>((const TT*)q, (const TT*)k, (const TT*)v, g, beta, state,      \
+                                                    (TT*)out, B * H, dv, scale)
   if (dk == 128) {
-    if (dtype == BF16)
-      gdn_step_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                               (const __nv_bfloat16*)v, g, beta, state,
-                                                               (__nv_bfloat16*)out, B * H, dv, scale);
-    else
-      gdn_step_kernel<float, 128><<<grid, 256, 0, s>>>((const float*)q, (const float*)k, (const float*)v, g, beta,
-                                                       state, (float*)out, B * H, dv, scale);
+    if (dtype == BF16) {
+      if (r4) GDN_STEP(__nv_bfloat16, 128, 4); else GDN_STEP(__nv_bfloat16, 128, 1);
+    } else {
+      if (r4) GDN_STEP(float, 128, 4); else GDN_STEP(float, 128, 1);
+    }
   } else if (dk == 64) {
-    if (dtype == BF16)
-      gdn_step_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                              (const __nv_bfloat16*)v, g, beta, state,
-                                                              (__nv_bfloat16*)out, B * H, dv, scale);
-    else
-      gdn_step_kernel<float, 64><<<grid, 256, 0, s>>>((const float*)q, (const float*)k, (const float*)v, g, beta,
-                                                      state, (float*)out, B * H, dv, scale);
+    if (dtype == BF16) {
+      if (r4) GDN_STEP(__nv_bfloat16, 64, 4); else GDN_STEP(__nv_bfloat16, 64, 1);
+    } else {
+      if (r4) GDN_STEP(float, 64, 4); else GDN_STEP(float, 64, 1);
+    }
   } else {
     return cudaErrorNotSupported;
   }
+#undef GDN_STEP
   return cudaGetLastError();
 }
 

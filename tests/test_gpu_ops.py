@@ -289,6 +289,30 @@ def test_gdn_step_and_chunk_continue(cuda, dtype):
         assert rel_l2(to64(S[b]), S_ref) < TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("dk,dv,offset", [(64, 64, 0), (64, 64, 1), (128, 128, 0), (128, 128, 1)])
+def test_gdn_step_layouts(cuda, dtype, dk, dv, offset):
+    """One recurrent step for both state access paths: four rows per warp with 16/8-byte
+    accesses (aligned state) and the plain form (a state that starts 4 bytes past an
+    aligned address)."""
+    import looped_hybrid_attention_b200 as L
+    B, H = 3, 5
+    q, k, v, g, beta, S0 = _gdn_inputs(B, 1, H, dk, dv, dtype, seed=21)
+    n = B * H * dv * dk
+    buf = torch.zeros(n + offset, device=cuda)
+    S = buf[offset:].view(B, H, dv, dk)
+    S.copy_(S0)
+    out = torch.empty((B, H, dv), dtype=DT[dtype], device=cuda)
+    scale = 1.0 / np.sqrt(dk)
+    L.gdn_step(q[:, 0].contiguous(), k[:, 0].contiguous(), v[:, 0].contiguous(), g[:, 0].contiguous(),
+               beta[:, 0].contiguous(), S, out, scale)
+    for b in range(B):
+        o_ref, S_ref = ops.gdn_recurrent(to64(q[b]), to64(k[b]), to64(v[b]), to64(g[b]), to64(beta[b]),
+                                         to64(S0[b]), scale)
+        assert rel_l2(to64(out[b]), o_ref[0]) < TOL[dtype]
+        assert rel_l2(to64(S[b]), S_ref) < TOL[dtype]
+
+
 def test_gdn_special_cases(cuda):
     import looped_hybrid_attention_b200 as L
     B, T, H, dk = 1, 100, 2, 64
