@@ -34,8 +34,8 @@ def test_sinkhorn_fp32(cuda, n):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19), (4096, 1501), (4096, 4133), (256, 2050), (1024, 1100), (2048, 1057),
-                                  (8192, 1030)])
+@pytest.mark.parametrize("d,N", [(256, 37), (4096, 19), (4096, 64), (4096, 100), (4096, 1501), (4096, 4133),
+                                  (256, 2050), (1024, 1100), (2048, 1057), (8192, 1030)])
 def test_mhc_modes(cuda, dtype, d, N):
     import looped_hybrid_attention_b200 as L
     code = L.BF16 if dtype == "bf16" else L.F32
