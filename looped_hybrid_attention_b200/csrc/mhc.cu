@@ -382,12 +382,6 @@ __device__ __forceinline__ void bulk_s2peer(uint32_t dst, uint32_t src, uint32_t
                : "memory");
 }
 
-// 1-D bulk copy global -> this CTA's shared memory, completing on an mbarrier.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // Shared-memory plan of mhc_cluster_kernel.  Two token-block buffers (the block in use and
 // the next one, in flight).  Each holds the two streams' slices as S/64 runs of
