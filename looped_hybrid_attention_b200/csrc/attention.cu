@@ -38,7 +38,10 @@ cudaError_t rope_table(float2* tab, int T, int pos0, int rot, float base, cudaSt
   return cudaGetLastError();
 }
 
-template <typename T, int DH, bool VEC>
+// One warp per R heads of one token (all query heads or all key heads: R divides Hq and
+// Hkv), so R rows' loads are in flight together and the norm gain and the rotary table
+// entries are read once for them.
+template <typename T, int DH, bool VEC, int R>
 __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, int ld_p, const T* __restrict__ q_norm,
                                                       const T* __restrict__ k_norm, T* __restrict__ q_out,
                                                       T* __restrict__ k_cache, T* __restrict__ v_cache, int kv_cap,
@@ -46,40 +49,54 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
                                                       float eps, const float2* __restrict__ tab) {
   constexpr int PER = DH / 32;         // contiguous elements per lane (even: rotary pairs stay local)
   const int lane = threadIdx.x & 31;
-  const int heads = Hq + Hkv;
+  const int groups = (Hq + Hkv) / R;
   const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int b = blockIdx.y;
-  if (w >= (long)T_len * heads) return;
-  const int t = (int)(w / heads), hh = (int)(w % heads);
+  if (w >= (long)T_len * groups) return;
+  const int t = (int)(w / groups), hh0 = (int)(w % groups) * R;
   const long m = (long)b * T_len + t;
   const int pos = pos0 + t;
   const T* row = P + m * ld_p;
-  const bool is_q = hh < Hq;
-  const int kvh = hh - Hq;
-  const T* src = is_q ? row + hh * DH : row + 2 * Hq * DH + kvh * DH;
+  const bool is_q = hh0 < Hq;
+  const int kvh0 = hh0 - Hq;
+  const T* src = is_q ? row + hh0 * DH : row + 2 * Hq * DH + kvh0 * DH;
   const T* gain = is_q ? q_norm : k_norm;
   // VEC: rows 16-byte aligned, so each lane moves its PER elements as 8-element vectors
   constexpr bool V8 = VEC && PER % 8 == 0;
-  float x[PER], gn[PER];
+  float x[R][PER], gn[PER];
   if constexpr (V8) {
 #pragma unroll
-    for (int u = 0; u < PER; u += 8) {
-      load8(src + lane * PER + u, x + u);
-      load8(gain + lane * PER + u, gn + u);
-    }
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int u = 0; u < PER; u += 8) load8(src + r * DH + lane * PER + u, x[r] + u);
+#pragma unroll
+    for (int u = 0; u < PER; u += 8) load8(gain + lane * PER + u, gn + u);
   } else {
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      x[u] = ldf(src + lane * PER + u);
-      gn[u] = ldf(gain + lane * PER + u);
-    }
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int u = 0; u < PER; ++u) x[r][u] = ldf(src + r * DH + lane * PER + u);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) gn[u] = ldf(gain + lane * PER + u);
   }
-  float ss = 0.f;
+  float inv[R];
 #pragma unroll
-  for (int u = 0; u < PER; ++u) ss += x[u] * x[u];
-  const float inv = rsqrtf(warp_sum(ss) / (float)DH + eps);
+  for (int r = 0; r < R; ++r) {
+    float ss = 0.f;
 #pragma unroll
-  for (int u = 0; u < PER; ++u) x[u] = x[u] * inv * gn[u];
+    for (int u = 0; u < PER; ++u) ss += x[r][u] * x[r][u];
+    inv[r] = ss;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < R; ++r) inv[r] += __shfl_xor_sync(0xffffffffu, inv[r], o);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    inv[r] = rsqrtf(inv[r] / (float)DH + eps);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) x[r][u] = x[r][u] * inv[r] * gn[u];
+  }
   // rotary on dims [0, rot): pair (2j, 2j+1), angle pos * base^(-2j/rot), evaluated in fp64
 #pragma unroll
   for (int u = 0; u < PER; u += 2) {
@@ -100,34 +117,40 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
         c = (float)cs;
         s = (float)sn;
       }
-      const float a0 = x[u], a1 = x[u + 1];
-      x[u] = a0 * c - a1 * s;
-      x[u + 1] = a0 * s + a1 * c;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float a0 = x[r][u], a1 = x[r][u + 1];
+        x[r][u] = a0 * c - a1 * s;
+        x[r][u + 1] = a0 * s + a1 * c;
+      }
     }
   }
-  T* dst;
-  if (is_q) {
-    dst = q_out + (m * Hq + hh) * DH;
-  } else {
-    const long slot = (((long)b * Hkv + kvh) * kv_cap + pos) * DH;
-    dst = k_cache + slot;
-    const T* vs = row + 2 * Hq * DH + Hkv * DH + kvh * DH;
-    T* vd = v_cache + slot;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    T* dst;
+    if (is_q) {
+      dst = q_out + (m * Hq + hh0 + r) * DH;
+    } else {
+      const long slot = (((long)b * Hkv + kvh0 + r) * kv_cap + pos) * DH;
+      dst = k_cache + slot;
+      const T* vs = row + 2 * Hq * DH + Hkv * DH + (kvh0 + r) * DH;
+      T* vd = v_cache + slot;
+      if constexpr (V8) {
+#pragma unroll
+        for (int u = 0; u < PER; u += 16 / (int)sizeof(T))
+          *reinterpret_cast<uint4*>(vd + lane * PER + u) = *reinterpret_cast<const uint4*>(vs + lane * PER + u);
+      } else {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
+      }
+    }
     if constexpr (V8) {
 #pragma unroll
-      for (int u = 0; u < PER; u += 16 / (int)sizeof(T))
-        *reinterpret_cast<uint4*>(vd + lane * PER + u) = *reinterpret_cast<const uint4*>(vs + lane * PER + u);
+      for (int u = 0; u < PER; u += 8) store8(dst + lane * PER + u, x[r] + u);
     } else {
 #pragma unroll
-      for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
+      for (int u = 0; u < PER; ++u) stf(dst + lane * PER + u, x[r][u]);
     }
-  }
-  if constexpr (V8) {
-#pragma unroll
-    for (int u = 0; u < PER; u += 8) store8(dst + lane * PER + u, x + u);
-  } else {
-#pragma unroll
-    for (int u = 0; u < PER; ++u) stf(dst + lane * PER + u, x[u]);
   }
 }
 
@@ -137,18 +160,20 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
                     cudaStream_t s, const float2* rope_tab) {
   if (T == 0 || B == 0) return cudaSuccess;
   const int warps = 8;
-  dim3 grid((unsigned)(((long)T * (Hq + Hkv) + warps - 1) / warps), B);
   auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
   const int es = dtype == BF16 ? 2 : 4;
   const bool vec = al16(P) && al16(q_norm) && al16(k_norm) && al16(q_out) && al16(k_cache) && al16(v_cache) &&
                    ((long)ld_p * es) % 16 == 0;
+  const int R = (vec && Hq % 4 == 0 && Hkv % 4 == 0) ? 4 : 1;   // heads per warp
+  dim3 grid((unsigned)(((long)T * ((Hq + Hkv) / R) + warps - 1) / warps), B);
 #define FA_PREP(TT, DHV)                                                                                   \
   do {                                                                                                     \
-    if (vec) FA_PREP_V(TT, DHV, true);                                                                     \
-    else FA_PREP_V(TT, DHV, false);                                                                        \
+    if (R == 4) FA_PREP_V(TT, DHV, true, 4);                                                               \
+    else if (vec) FA_PREP_V(TT, DHV, true, 1);                                                             \
+    else FA_PREP_V(TT, DHV, false, 1);                                                                     \
   } while (0)
-#define FA_PREP_V(TT, DHV, V)                                                                              \
-  fa_prep_kernel<TT, DHV, V><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,            \
+#define FA_PREP_V(TT, DHV, V, RR)                                                                          \
+  fa_prep_kernel<TT, DHV, V, RR><<<grid, warps * 32, 0, s>>>((const TT*)P, ld_p, (const TT*)q_norm,            \
                                                       (const TT*)k_norm, (TT*)q_out, (TT*)k_cache,         \
                                                       (TT*)v_cache, kv_cap, T, pos0, Hq, Hkv, rotary_dims, \
                                                       rope_base, eps, rope_tab)

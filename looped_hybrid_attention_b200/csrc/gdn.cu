@@ -64,40 +64,59 @@ __global__ void gdn_prep_kernel(const T* __restrict__ P, int ld_p, const float* 
   }
 }
 
-// bf16, dk = dv = 128, 16-byte aligned rows: one warp per (token, head) with 16-byte
-// vectors -- lanes 0-15 normalise q, lanes 16-31 normalise k (8 elements each, sums
-// reduced within each half-warp), lanes 0-15 copy v.
+// bf16, dk = dv = 128, 16-byte aligned rows: one warp per R heads of one token with
+// 16-byte vectors -- lanes 0-15 normalise q, lanes 16-31 normalise k (8 elements each,
+// sums reduced within each half-warp), lanes 0-15 copy v; all R heads' loads are in
+// flight together.
+template <int R>
 __global__ void gdn_prep_v128_kernel(const __nv_bfloat16* __restrict__ P, int ld_p, const float* __restrict__ a_bias,
                                      const float* __restrict__ b_bias, __nv_bfloat16* __restrict__ q,
                                      __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
                                      float* __restrict__ g, float* __restrict__ beta, int M, int H, float eps) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
+  const int groups = H / R;
   const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (w >= (long)M * H) return;
-  const long m = w / H;
-  const int h = (int)(w % H);
+  if (w >= (long)M * groups) return;
+  const long m = w / groups;
+  const int h0 = (int)(w % groups) * R;
   const __nv_bfloat16* row = P + m * ld_p;
-  const __nv_bfloat16* src = row + half * H * D + h * D + hl * 8;     // q (half 0) or k (half 1)
-  float x[8];
-  load8(src, x);
-  float ss = 0.f;
+  float x[R][8];
+  uint4 vv[R];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
+  for (int r = 0; r < R; ++r) load8(row + half * H * D + (h0 + r) * D + hl * 8, x[r]);   // q (half 0) or k
+  if (!half) {
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float inv = rsqrtf(ss + eps);
+    for (int r = 0; r < R; ++r) vv[r] = *reinterpret_cast<const uint4*>(row + 2 * H * D + (h0 + r) * D + hl * 8);
+  }
+  float ss[R];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] *= inv;
-  store8((half ? k : q) + w * D + hl * 8, x);
-  if (!half)
-    *reinterpret_cast<uint4*>(v + w * D + hl * 8) = *reinterpret_cast<const uint4*>(row + 2 * H * D + h * D + hl * 8);
-  if (lane == 16) {
+  for (int r = 0; r < R; ++r) {
+    ss[r] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss[r] += x[r][i] * x[r][i];
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < R; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], o);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float inv = rsqrtf(ss[r] + eps);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[r][i] *= inv;
+    const long wr = m * H + h0 + r;
+    store8((half ? k : q) + wr * D + hl * 8, x[r]);
+    if (!half) *reinterpret_cast<uint4*>(v + wr * D + hl * 8) = vv[r];
+  }
+  if (lane >= 16 && lane < 16 + R) {
+    const int h = h0 + lane - 16;
+    const long wr = m * H + h;
     const float a = __bfloat162float(row[2 * H * D + H * D + h]) + a_bias[h];
     const float b = __bfloat162float(row[2 * H * D + H * D + H + h]) + b_bias[h];
     const float sp = a > 20.f ? a : log1pf(expf(a));    // softplus
-    g[w] = -sp;
-    beta[w] = 1.f / (1.f + expf(-b));
+    g[wr] = -sp;
+    beta[wr] = 1.f / (1.f + expf(-b));
   }
 }
 
@@ -109,9 +128,16 @@ cudaError_t gdn_prep(const void* P, int ld_p, const float* a_bias, const float* 
   dim3 grid((unsigned)(((long)M * H + warps - 1) / warps));
   auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
   if (dtype == BF16 && dk == 128 && dv == 128 && ld_p % 8 == 0 && al16(P) && al16(q) && al16(k) && al16(v)) {
-    gdn_prep_v128_kernel<<<grid, warps * 32, 0, s>>>((const __nv_bfloat16*)P, ld_p, a_bias, b_bias,
-                                                     (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, g,
-                                                     beta, M, H, eps);
+    if (H % 4 == 0) {                             // four heads per warp
+      const dim3 g4((unsigned)(((long)M * (H / 4) + warps - 1) / warps));
+      gdn_prep_v128_kernel<4><<<g4, warps * 32, 0, s>>>((const __nv_bfloat16*)P, ld_p, a_bias, b_bias,
+                                                        (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, g,
+                                                        beta, M, H, eps);
+    } else {
+      gdn_prep_v128_kernel<1><<<grid, warps * 32, 0, s>>>((const __nv_bfloat16*)P, ld_p, a_bias, b_bias,
+                                                          (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v,
+                                                          g, beta, M, H, eps);
+    }
     return cudaGetLastError();
   }
   if (dtype == BF16)

@@ -329,9 +329,11 @@ def test_gdn_special_cases(cuda):
     assert torch.equal(S, S0)
 
 
-def test_gdn_prep(cuda):
+@pytest.mark.parametrize("H", [16, 6])
+def test_gdn_prep(cuda, H):
+    """Four heads per warp (H % 4 == 0) and one (H = 6)."""
     import looped_hybrid_attention_b200 as L
-    M, H, dk, dv = 50, 16, 128, 128
+    M, dk, dv = 50, 128, 128
     n_in = 2 * H * dk + H * dv + 2 * H
     P = rnd((M, n_in), 20, "P", dtype="bf16")
     ab, bb = rnd((H,), 21, "ab"), rnd((H,), 22, "bb")
