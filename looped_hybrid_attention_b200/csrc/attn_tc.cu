@@ -54,6 +54,23 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Two fp32 FMAs / adds as one packed instruction (each lane rounds exactly as fmaf / +).
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                       float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __global__ void __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __nv_bfloat16* __restrict__ q, int ld_q, const __grid_constant__ CUtensorMap tK,
                    const __grid_constant__ CUtensorMap tV, const __nv_bfloat16* __restrict__ gate, int ld_gate,
@@ -297,16 +314,19 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       // this half's 64 keys of P as bf16 pairs (key 2i in the low half of column i) into
       // columns [32 half, 32 half + 32) of this tile's S buffer, the A operand of P V
-      float psum = 0.f;
+      // (packed f32x2 FMAs and adds: two scores per instruction)
+      float ps0 = 0.f, ps1 = 0.f;
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2(fmaf(t[2 * i], scale_log2, -m_used));
-        const float p1 = ex2(fmaf(t[2 * i + 1], scale_log2, -m_used));
-        psum += p0 + p1;
+        float x0, x1;
+        fma_x2(x0, x1, t[2 * i], t[2 * i + 1], scale_log2, scale_log2, -m_used, -m_used);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        add_x2(ps0, ps1, ps0, ps1, p0, p1);
         const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
         w[i] = *reinterpret_cast<const uint32_t*>(&pr);
       }
+      const float psum = ps0 + ps1;
       tmem_st32(tmem + lane_off + s * AT_N + half * 32, w);
       tmem_wait_st();
       l += psum;
