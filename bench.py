@@ -118,6 +118,7 @@ def oracle_sample(T=64, seed=0):
 
 
 def cpu_cores():
+    """Threads the oracle's numpy BLAS uses (what the all-core number ran on)."""
     try:
         import threadpoolctl
         info = threadpoolctl.threadpool_info()
@@ -127,13 +128,35 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+SAMPLE_CAVEATS = ("scaled from one group's 4 executions to 56 per token: the sample's attention rows are "
+                  "64 keys long, so the quadratic attention cost of an 8,192-token prefill is under-counted, "
+                  "and the LM head is left out")
+
+
 def cpu_baseline_entry(T=64):
+    """The oracle on the bounded sample, once on all host cores and once on one core."""
+    import threadpoolctl
     dt, tokens, execs = oracle_sample(T)
+    with threadpoolctl.threadpool_limits(limits=1):
+        dt1, _, _ = oracle_sample(T)
     # per-token time of the full stack = (time per execution per token) x 56 executions
-    per_token = dt / tokens / execs * 56
+    per_token, per_token1 = dt / tokens / execs * 56, dt1 / tokens / execs * 56
     return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "single_core": {"value": 1.0 / per_token1, "unit": "tokens/s", "cores": 1, "sample_s": round(dt1, 3)},
             "sample": f"oracle forward of one full-width group (3 GDN + 1 GQA + mHC, d 4096) on {tokens} tokens "
-                      f"({dt:.2f} s), scaled to 56 executions per token; LM head excluded"}
+                      f"({dt:.2f} s on {cpu_cores()} BLAS threads, {dt1:.2f} s on one); " + SAMPLE_CAVEATS}
 
 
 def dist_setup():
@@ -178,19 +201,27 @@ def run_reference(args, world, rank):
         return
     for _ in range(args.warmup):
         oracle_sample(args.ref_tokens)
-    times = []
+    times, sample_s = [], []
     for _ in range(args.steps):
         dt, tokens, execs = oracle_sample(args.ref_tokens)
+        sample_s.append(dt)
         times.append(dt / tokens / execs * 56)
     value = 1.0 / (sum(times) / len(times))
+    # a step is one bounded sample: ms_per_step is the time actually measured for it; the
+    # tokens/s value is extrapolated from it to the 56-execution stack
     line = {"impl": "reference", "metric": "prefill tokens/s (56-execution looped hybrid stack)", "value": value,
             "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000.0 * sum(times) / len(times) * SEQ, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": round(1000.0 * sum(sample_s) / len(sample_s), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": SEQ, "parallelism": "cpu oracle"},
+            "step": f"one oracle forward of one full-width group (3 GDN + 1 GQA + mHC, d 4096) on "
+                    f"{args.ref_tokens} tokens; ms_per_step is that sample's measured time",
+            "extrapolated": {"value_from": "seconds per token per execution x 56 executions", "caveats": SAMPLE_CAVEATS,
+                             "ms_per_8192_token_prefill": round(1000.0 * sum(times) / len(times) * SEQ, 1)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                             "nproc": os.cpu_count(), "cpu_model": cpu_model(),
                              "sample": f"each step: oracle forward of one full-width group on {args.ref_tokens} "
-                                       "tokens, scaled to 56 executions per token"},
+                                       "tokens, scaled to 56 executions per token; " + SAMPLE_CAVEATS},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -242,6 +273,15 @@ def summarize(kernels, steps, peaks, sustained=True, tensor_bound=("gemm", "atte
             e["gbs"] = round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)
         per_kernel[kname] = e
     return roof, per_kernel
+
+
+def step_tensor_roofline(kernels, ms_step, peaks):
+    """The whole prefill step against the tensor roofline: every kernel's algorithmic FLOPs of
+    one step over the step's time, as a fraction of the sustained bf16 peak."""
+    flops = sum(v["flops"] for v in kernels.values())
+    achieved = flops / (ms_step / 1e3) / 1e12
+    return {"bound": "tensor", "algorithmic_flops_per_step": flops, "achieved_tflops": round(achieved, 1),
+            "peak": peaks["bf16_tflops_sustained"], "frac": round(achieved / peaks["bf16_tflops_sustained"], 4)}
 
 
 def profiled(m, fn, n):
@@ -406,7 +446,8 @@ def run_long(args, m, s, dev, world, seed):
            "device_bytes_in_use": total - free,
            "gpu_launches": sum(v["launches"] for v in kernels.values()) * args.long_steps,
            "kernel_table_steps": 1,
-           "roofline": roof, "kernels": per_kernel, "clocks": clk.summary()}
+           "roofline": roof, "step_roofline": step_tensor_roofline(kernels, ms / args.long_steps, load_peaks()),
+           "kernels": per_kernel, "clocks": clk.summary()}
     del c
     return out
 
@@ -484,8 +525,9 @@ def run_ours(args, world, rank, local):
                        "l2": "inputs larger than L2 (16.3 GB of weights streamed per step)"},
             "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": ids.numel() * 4, "d2h_bytes_per_step": logits.numel() * 4},
-            "gpu_launches": launches, "kernel_table_steps": 1, "roofline": roof, "kernels": per_kernel,
-            "clocks": clk.summary()}
+            "gpu_launches": launches, "kernel_table_steps": 1, "roofline": roof,
+            "step_roofline": step_tensor_roofline(kernels, ms / args.steps, peaks),
+            "kernels": per_kernel, "clocks": clk.summary()}
     if not args.no_decode or not args.no_long:
         del c
         torch.cuda.empty_cache()
@@ -497,6 +539,21 @@ def run_ours(args, world, rank, local):
         return
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_entry(args.ref_tokens)
+    # compact per-leg summary as the line's last key, so that a reader of the line's tail
+    # sees every leg's number after the long per-kernel tables
+    legs = {"prefill": {"value": line["value"], "unit": "tokens/s", "ms_per_step": line["ms_per_step"],
+                        "roofline_kernel": roof["kernel"], "roofline_frac": roof["frac"],
+                        "step_frac_of_tensor_roofline": line["step_roofline"]["frac"],
+                        "sm_mhz": line["clocks"]["sm_mhz"]}}
+    for key in ("decode", "long_prefill"):
+        if key in line:
+            leg = line[key]
+            legs[key] = {"value": leg["value"], "unit": leg["unit"], "ms_per_step": leg["ms_per_step"],
+                         "roofline_kernel": leg["roofline"]["kernel"], "roofline_frac": leg["roofline"]["frac"],
+                         "sm_mhz": leg["clocks"]["sm_mhz"]}
+            if "step_roofline" in leg:
+                legs[key]["step_frac_of_hbm_roofline"] = leg["step_roofline"]["frac"]
+    line["legs"] = legs
     print(json.dumps(line), flush=True)
 
 

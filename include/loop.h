@@ -161,6 +161,21 @@ loop_status loop_forward_hidden(loop_model* m, loop_cache* c, const void* h_in, 
 loop_status loop_decode_step(loop_model* m, loop_cache* c, const int32_t* tok, float* logits,
                              int32_t* next_tok, void* stream);
 
+/* Hidden-state taps ("原地套圈" investigation §03: the draft models read the target's
+ * hidden states at execution indices [3, 27, 51, 53, 54] -- the end of the head, of the
+ * first and second loop pass, and two tail layers).  While taps are set, every
+ * loop_prefill / loop_forward_hidden / loop_decode_step of this model also writes, for
+ * i < n, the hidden state of its new tokens after execution exec[i] to out[i]
+ * ([B*T, d] dtype, device, caller-owned, rows in token-major order): outside the loop
+ * block the layer's output h; inside it the mean of the two residual streams after that
+ * execution's mix, (X'_0 + X'_1) / 2.  max_rows is the row capacity of every buffer: a
+ * call with more than max_rows new tokens returns LOOP_ERR_CAPACITY and launches nothing.
+ * exec[i] must lie in [0, n_executions) and be distinct (LOOP_ERR_INVALID_ARG).  n = 0
+ * clears the taps.  exec and out are host arrays, copied; the buffers must stay valid
+ * while set. */
+loop_status loop_set_taps(loop_model* m, int n, const int32_t* exec /* host [n] */,
+                          void* const* out /* host [n] of device pointers */, long max_rows);
+
 /* ---------------------------------------------------------------- per-op entry points
  * All pointers device, caller-owned, contiguous unless a row stride is given.  */
 
@@ -173,8 +188,9 @@ loop_status loop_decode_step(loop_model* m, loop_cache* c, const int32_t* tok, f
  * out [B, T, H, dv] dtype.  Supported: (dk, dv) in {(64,64), (128,128)}, chunk 64.
  * workspace: device scratch of loop_gdn_workspace_bytes(B, T, H, dk, dv) bytes for the
  * two-pass scan (every chunk's intra-chunk solve in parallel, then the sequential state
- * pass), or NULL for a single-pass kernel that needs no scratch (slower).  Calls that
- * share a workspace must not overlap on the GPU. */
+ * pass), or NULL for a single-pass kernel that needs no scratch (slower).  With a
+ * workspace, q, k, v and the workspace must be 16-byte aligned (LOOP_ERR_UNSUPPORTED
+ * otherwise).  Calls that share a workspace must not overlap on the GPU. */
 loop_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* out, int B, int T, int H,
                           int dk, int dv, int chunk, float scale, void* workspace, int dtype,
@@ -204,7 +220,13 @@ loop_status gdn_prep(const void* P, int ld_p, const float* a_bias, const float* 
  * (per-execution slab layout; kv_cap >= Tkv); out [B, Tq, Hq, dh] contiguous.
  * q and k are used as given (already QK-normed and rotated).
  * workspace: device scratch of loop_gqa_workspace_bytes(...) bytes, or NULL (then a
- * single pass over the keys is used). */
+ * single pass over the keys is used).
+ * Kernels by shape: bf16 with Tq >= 16, dh 256 and 128 % (Hq/Hkv) == 0 runs the tcgen05
+ * flash kernel; bf16 with Tq == 1 runs a flash-decode kernel (dh 128/256 with <= 16, dh 64
+ * with <= 4 q heads per KV head); other calls run one warp per query row.  The tiled kernels
+ * need 16-byte aligned q, k, v, gate and row strides that are multiples of 8 elements: a
+ * call whose shape selects one of them with buffers that are not is refused with
+ * LOOP_ERR_UNSUPPORTED (never run on a slower kernel). */
 loop_status gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
                      const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype, void* stream);
@@ -216,8 +238,11 @@ size_t loop_gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
  * loop that must not take the implicit device synchronisation of cudaMalloc/cudaFree.
  * Same arguments and result as gqa_attn (minus `workspace`); the split-K scratch is a
  * fixed 32 MiB array in the library's device memory, held on every GPU that loads the
- * library until the process exits.  A problem whose scratch (loop_gqa_workspace_bytes)
- * exceeds 32 MiB is rejected with LOOP_ERR_CAPACITY and nothing is launched.  The first
+ * library until the process exits.  A problem whose scratch exceeds 32 MiB is rejected
+ * with LOOP_ERR_CAPACITY and nothing is launched; the scratch is the split-K partials of the
+ * kernel that the call's shape selects, B*Tq*Hq*splits*(dh+2)*4 bytes when that kernel
+ * splits the keys (single-token decode, the row kernel) and none otherwise (bf16 multi-token
+ * queries with head dim 256); it never exceeds loop_gqa_workspace_bytes.  The first
  * call on each device (with that device current) looks the array's address up with
  * cudaGetSymbolAddress; make that first call before any stream capture.  Every call
  * shares the array: calls that overlap on the GPU (different streams, or different host
@@ -266,7 +291,9 @@ loop_status sinkhorn_fp32(const float* logits, float* out, int N, int n, int ite
  *   1 ADD:    Y = X W^T + R, R [M, N] (row stride ldr) may alias Y
  *   2 SWIGLU: Y [M, N] = silu(X W^T) * (X W2^T), W2 [N, K] (the FFN's up map)
  *   3 F32:    Y [M, N] fp32
- * K must be a multiple of 8 for bf16.
+ * K must be a multiple of 8 for bf16, and bf16 calls need 16-byte aligned X, W (W2) and
+ * a row stride ldx that is a multiple of 8 (TMA); otherwise LOOP_ERR_UNSUPPORTED (bf16 has
+ * no slower fallback kernel).
  * bf16 calls with M <= 128 (decode batches, a last position) stream W through every SM
  * with the batch as the MMA's N dimension.
  * workspace: optional device scratch of loop_linear_workspace_bytes(M, N, K, epilogue)

@@ -77,6 +77,7 @@ _SIGS = {
     "loop_prefill": ([_P, _P, _P, _I, _I, _P, _P], _I),
     "loop_forward_hidden": ([_P, _P, _P, _P, _I, _I, _P], _I),
     "loop_decode_step": ([_P, _P, _P, _P, _P, _P], _I),
+    "loop_set_taps": ([_P, _I, _P, _P, ctypes.c_long], _I),
     "gdn_chunk_fwd": ([_P] * 7 + [_I] * 6 + [_F, _P, _I, _P], _I),
     "loop_gdn_workspace_bytes": ([_I] * 5, _Z),
     "gdn_step": ([_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
@@ -236,6 +237,14 @@ class Model:
     def decode_step(self, cache, tok, logits, next_tok, stream=None):
         check(_lib.loop_decode_step(self.handle, cache.handle, ptr(tok), ptr(logits), ptr(next_tok),
                                     _stream(stream)), "loop_decode_step")
+
+    def set_taps(self, execs, outs, max_rows):
+        """Hidden-state taps after the given executions into the given [rows, d] device tensors ([] clears)."""
+        n = len(execs)
+        ex = (ctypes.c_int32 * max(n, 1))(*execs)
+        ps = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in outs])
+        check(_lib.loop_set_taps(self.handle, n, ex, ps, max_rows), "loop_set_taps")
+        self._taps = list(outs)           # keep the buffers alive while set
 
 
 class Cache:

@@ -738,9 +738,37 @@ size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
   return (size_t)B * Tq * Hq * s * (dh + 2) * sizeof(float);
 }
 
-int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace) {
-  if (Tq >= 16) return 1;
-  return has_workspace && attn_splits(B, Tq, Tkv, Hkv) > 1 ? 2 : 1;
+// Which kernel a call runs, from its shape alone:
+//   ATT_TC      multi-token queries, bf16, head dim 256, 128 % (Hq/Hkv) == 0: attn_tc.cu
+//   ATT_DEC_TC  one query token, bf16, head dim 128/256, <= 16 q heads per KV head: tensor-core flash-decode
+//   ATT_DEC     one query token, bf16, head dim 64, <= 4 q heads per KV head: flash-decode
+//   ATT_ROWS    everything else (fp32 models; bf16 prefill segments of 2..15 tokens, head dims without
+//               a tiled kernel): one warp per query row
+enum AttnPath { ATT_TC, ATT_DEC_TC, ATT_DEC, ATT_ROWS };
+
+static AttnPath attn_path(int Tq, int dtype, int dh, int Hq, int Hkv) {
+  const int rep = Hq / Hkv;
+  if (dtype == BF16 && Tq >= 16 && dh == 256 && 128 % rep == 0) return ATT_TC;   // 128 MMA rows = rep heads x positions
+  if (dtype == BF16 && Tq == 1 && (dh == 256 || dh == 128) && rep <= 16) return ATT_DEC_TC;
+  if (dtype == BF16 && Tq == 1 && dh == 64 && rep <= 4) return ATT_DEC;
+  return ATT_ROWS;
+}
+
+// Key splits (> 1 means a second, combining launch and scratch partials) of a call given a workspace.
+static int attn_path_splits(AttnPath p, int B, int Tq, int Tkv, int Hkv) {
+  if (p == ATT_TC) return 1;
+  return attn_splits(B, p == ATT_ROWS ? Tq : 1, Tkv, Hkv);
+}
+
+size_t gqa_scratch_bytes(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype) {
+  if (B <= 0 || Tq <= 0 || Tkv <= 0) return 0;
+  const int n = attn_path_splits(attn_path(Tq, dtype, dh, Hq, Hkv), B, Tq, Tkv, Hkv);
+  return n > 1 ? (size_t)B * Tq * Hq * n * (dh + 2) * sizeof(float) : 0;
+}
+
+int gqa_launches(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype, bool has_workspace) {
+  const AttnPath p = attn_path(Tq, dtype, dh, Hq, Hkv);
+  return has_workspace && attn_path_splits(p, B, Tq, Tkv, Hkv) > 1 ? 2 : 1;
 }
 
 bool gqa_supported(int dh, int Hq, int Hkv) {
@@ -772,25 +800,23 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
                      cudaStream_t s) {
   if (B == 0 || Tq == 0) return cudaSuccess;
-  // multi-token queries (prefill) go to the tensor-core kernel; single-token decode keeps
-  // the split-K kernel, which streams the KV slab at full width
-  if (Tq >= 16 && Tkv > 0 && gqa_tc_supported(dh, dtype, q, ld_q, gate, ld_gate, k, v, kv_cap)) {
-    cudaError_t e = gqa_attn_tc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, s);
-    if (e != cudaErrorNotSupported) return e;
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  const AttnPath path = attn_path(Tq, dtype, dh, Hq, Hkv);
+  // The tiled kernels move 16-byte pieces (TMA boxes, cp.async); a call whose shape selects one of
+  // them but whose buffers are not 16-byte aligned is refused rather than run on a slower kernel.
+  if (path == ATT_TC) {
+    if (Tkv == 0) return cudaSuccess;
+    if (!gqa_tc_supported(dh, dtype, q, ld_q, gate, ld_gate, k, v, kv_cap)) return cudaErrorNotSupported;
+    return gqa_attn_tc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, s);
   }
-  // single-token decode (bf16, <= 4 q heads per KV head): the tiled flash-decode kernel
-  if (Tq == 1 && dtype == BF16 && Hq / Hkv <= 16 && (dh == 256 || dh == 128) && ((uintptr_t)k % 16 == 0) &&
-      ((uintptr_t)v % 16 == 0) && ((uintptr_t)q % 16 == 0) && ld_q % 8 == 0) {
+  if (path == ATT_DEC_TC) {
+    if (!(al16(k) && al16(v) && al16(q) && ld_q % 8 == 0)) return cudaErrorNotSupported;
     if (dh == 256)
       return launch_decode_tc<256>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
     return launch_decode_tc<128>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
   }
-  if (Tq == 1 && dtype == BF16 && Hq / Hkv <= 4 && (dh == 256 || dh == 128 || dh == 64) &&
-      ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0)) {
-    if (dh == 256)
-      return launch_decode<256>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
-    if (dh == 128)
-      return launch_decode<128>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
+  if (path == ATT_DEC) {
+    if (!(al16(k) && al16(v))) return cudaErrorNotSupported;
     return launch_decode<64>(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tkv, q_off, Hq, Hkv, causal, workspace, s);
   }
 #define ATTN(TT, DHV) \

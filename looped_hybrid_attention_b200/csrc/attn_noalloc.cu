@@ -49,23 +49,19 @@ loop_status scratch_address(void** out) {
 extern "C" loop_status gqa_attn_noalloc(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
                                         const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                                         int Hq, int Hkv, int dh, int causal, int dtype, void* stream) {
-  if (dtype != LOOP_F32 && dtype != LOOP_BF16) return fail(LOOP_ERR_INVALID_ARG, "gqa_attn_noalloc: bad dtype");
-  if (B < 0 || Tq < 0 || Tkv < 0 || q_off < 0) return fail(LOOP_ERR_INVALID_ARG, "gqa_attn_noalloc: negative size");
-  if (B == 0 || Tq == 0) return LOOP_OK;
-  if (!q || !k || !v || !out) return fail(LOOP_ERR_INVALID_ARG, "gqa_attn_noalloc: NULL argument");
-  if (!lk::gqa_supported(dh, Hq, Hkv))
-    return fail(LOOP_ERR_UNSUPPORTED, "gqa_attn_noalloc: head dim or head ratio not supported");
-  if (kv_cap < Tkv) return fail(LOOP_ERR_SHAPE, "gqa_attn_noalloc: kv_cap < Tkv");
-  if (ld_q < Hq * dh || (gate && ld_gate < Hq * dh))
-    return fail(LOOP_ERR_SHAPE, "gqa_attn_noalloc: row stride smaller than Hq*dh");
-  if (causal && q_off + Tq > Tkv) return fail(LOOP_ERR_SHAPE, "gqa_attn_noalloc: causal needs q_off + Tq <= Tkv");
-  const size_t need = lk::gqa_workspace_bytes(B, Tq, Tkv, Hq, dh);
+  bool empty = false;
+  loop_status st = gqa_check_args("gqa_attn_noalloc", q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off,
+                                  Hq, Hkv, dh, causal, dtype, &empty);
+  if (st != LOOP_OK || empty) return st;
+  // The scratch this call's kernels use: the split-K partials of the kernel that its shape
+  // selects, at that kernel's split count (0 for kernels without partials).
+  const size_t need = lk::gqa_scratch_bytes(B, Tq, Tkv, Hq, Hkv, dh, dtype);
   if (need > kScratchBytes)
     return fail(LOOP_ERR_CAPACITY, "gqa_attn_noalloc: this problem needs " + std::to_string(need) +
                                        " bytes of scratch but the built-in scratch holds " +
                                        std::to_string(kScratchBytes) + " (32 MiB); use gqa_attn with a workspace");
   void* scratch = nullptr;
-  loop_status st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != LOOP_OK) return st;
   // Every (row, head, split) slot of the scratch is written before it is read, so the
   // previous call's contents never leak into this one and nothing needs clearing.

@@ -22,6 +22,25 @@ static loop_status launched(cudaError_t e, const char* what) {
 static bool dtype_ok(int dt) { return dt == LOOP_F32 || dt == LOOP_BF16; }
 static cudaStream_t S(void* s) { return (cudaStream_t)s; }
 
+loop_status gqa_check_args(const char* who, const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                           const void* gate, int ld_gate, const void* out, int B, int Tq, int Tkv, int q_off, int Hq,
+                           int Hkv, int dh, int causal, int dtype, bool* empty) {
+  const std::string w = std::string(who) + ": ";
+  *empty = false;
+  if (!dtype_ok(dtype)) return fail(LOOP_ERR_INVALID_ARG, w + "bad dtype");
+  if (B < 0 || Tq < 0 || Tkv < 0 || q_off < 0) return fail(LOOP_ERR_INVALID_ARG, w + "negative size");
+  if (B == 0 || Tq == 0) {
+    *empty = true;
+    return LOOP_OK;
+  }
+  if (!q || !k || !v || !out) return fail(LOOP_ERR_INVALID_ARG, w + "NULL argument");
+  if (!gqa_supported(dh, Hq, Hkv)) return fail(LOOP_ERR_UNSUPPORTED, w + "head dim or head ratio not supported");
+  if (kv_cap < Tkv) return fail(LOOP_ERR_SHAPE, w + "kv_cap < Tkv");
+  if (ld_q < Hq * dh || (gate && ld_gate < Hq * dh)) return fail(LOOP_ERR_SHAPE, w + "row stride smaller than Hq*dh");
+  if (causal && q_off + Tq > Tkv) return fail(LOOP_ERR_SHAPE, w + "causal attention needs q_off + Tq <= Tkv");
+  return LOOP_OK;
+}
+
 extern "C" {
 
 const char* loop_version(void) { return "loop-b200 0.1 (sm_100a)"; }
@@ -222,6 +241,23 @@ loop_status loop_decode_step(loop_model* m, loop_cache* c, const int32_t* tok, f
   return run_decode(m, c, tok, logits, next_tok, S(stream));
 }
 
+loop_status loop_set_taps(loop_model* m, int n, const int32_t* exec, void* const* out, long max_rows) {
+  REQUIRE(m, LOOP_ERR_INVALID_ARG, "model is NULL");
+  REQUIRE(n >= 0 && max_rows >= 0, LOOP_ERR_INVALID_ARG, "n and max_rows must be >= 0");
+  REQUIRE(n == 0 || (exec && out), LOOP_ERR_INVALID_ARG, "exec or out is NULL");
+  const int n_exec = (int)m->sched.size();
+  for (int i = 0; i < n; ++i) {
+    REQUIRE(exec[i] >= 0 && exec[i] < n_exec, LOOP_ERR_INVALID_ARG,
+            "tap execution index " + std::to_string(exec[i]) + " outside [0, " + std::to_string(n_exec) + ")");
+    REQUIRE(out[i], LOOP_ERR_INVALID_ARG, "tap buffer is NULL");
+    for (int j = 0; j < i; ++j) REQUIRE(exec[j] != exec[i], LOOP_ERR_INVALID_ARG, "execution tapped twice");
+  }
+  m->tap_exec.assign(exec, exec + n);
+  m->tap_out.assign(out, out + n);
+  m->tap_rows = n ? max_rows : 0;
+  return LOOP_OK;
+}
+
 // ------------------------------------------------------------------ per-op entry points
 size_t loop_gdn_workspace_bytes(int B, int T, int H, int dk, int dv) {
   if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
@@ -270,14 +306,10 @@ size_t loop_gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh) {
 loop_status gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate, int ld_gate,
                      void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int dh, int causal,
                      void* workspace, int dtype, void* stream) {
-  REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
-  REQUIRE(B >= 0 && Tq >= 0 && Tkv >= 0 && q_off >= 0, LOOP_ERR_INVALID_ARG, "negative size");
-  if (B == 0 || Tq == 0) return LOOP_OK;
-  REQUIRE(q && k && v && out, LOOP_ERR_INVALID_ARG, "NULL argument");
-  REQUIRE(gqa_supported(dh, Hq, Hkv), LOOP_ERR_UNSUPPORTED, "head dim or head ratio not supported");
-  REQUIRE(kv_cap >= Tkv, LOOP_ERR_SHAPE, "kv_cap < Tkv");
-  REQUIRE(ld_q >= Hq * dh && (!gate || ld_gate >= Hq * dh), LOOP_ERR_SHAPE, "row stride smaller than Hq*dh");
-  REQUIRE(!causal || q_off + Tq <= Tkv, LOOP_ERR_SHAPE, "causal attention needs q_off + Tq <= Tkv");
+  bool empty = false;
+  loop_status st = gqa_check_args("gqa_attn", q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, dh,
+                                  causal, dtype, &empty);
+  if (st != LOOP_OK || empty) return st;
   return launched(lk::gqa_attn(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, dh, causal,
                                workspace, dtype, S(stream)),
                   "gqa_attn");

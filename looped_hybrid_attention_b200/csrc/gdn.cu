@@ -1186,7 +1186,7 @@ cudaError_t gdn_chunk(const void* q, const void* k, const void* v, const float* 
   if (T == 0 || B == 0) return cudaSuccess;
   // the two-pass kernels copy 16-byte pieces of q, k, v rows and of the workspace
   auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
-  if (workspace && !(al16(q) && al16(k) && al16(v) && al16(workspace))) workspace = nullptr;
+  if (workspace && !(al16(q) && al16(k) && al16(v) && al16(workspace))) return cudaErrorNotSupported;
   if (workspace) {
     if (dk == 128 && dv == 128)
       return dtype == BF16

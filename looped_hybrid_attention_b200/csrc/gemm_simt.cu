@@ -98,10 +98,9 @@ cudaError_t linear_simt(const void* X, int ldx, const void* W, const void* W2, c
 cudaError_t linear(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr,
                    void* Y, int ldy, int M, int N, int K, int epi, int dtype, cudaStream_t s, void* ws,
                    size_t ws_bytes) {
-  if (dtype == BF16) {
-    cudaError_t e = linear_tc(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, s, ws, ws_bytes);
-    if (e != cudaErrorNotSupported) return e;
-  }
+  // bf16 runs on the tensor cores only: a shape or alignment the tcgen05 kernels do not
+  // take is an error (cudaErrorNotSupported), never a silent detour to the FP32 SIMT kernel.
+  if (dtype == BF16) return linear_tc(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, s, ws, ws_bytes);
   return linear_simt(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, epi, dtype, s);
 }
 

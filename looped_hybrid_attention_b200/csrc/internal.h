@@ -63,9 +63,12 @@ cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                      const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
                      cudaStream_t s);
+// Workspace bound for any Hkv and dtype (what loop_gqa_workspace_bytes promises).
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
+// Exact scratch bytes gqa_attn uses with a workspace for this call's shape (0: none).
+size_t gqa_scratch_bytes(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype);
 bool gqa_supported(int dh, int Hq, int Hkv);
-int gqa_launches(int B, int Tq, int Tkv, int Hkv, bool has_workspace);
+int gqa_launches(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype, bool has_workspace);
 // tcgen05 flash attention (bf16, head dim 256); used for multi-token queries.
 bool gqa_tc_supported(int dh, int dtype, const void* q, int ld_q, const void* gate, int ld_gate, const void* k,
                       const void* v, int kv_cap);

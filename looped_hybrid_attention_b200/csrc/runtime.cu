@@ -133,7 +133,7 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->F, M * d * es},
       {&m->coeffs, M * 8 * sizeof(float)},
       {&m->rope, (size_t)Tq * (c.rotary_dims / 2) * sizeof(float2)},
-      {&m->attn_ws, gqa_workspace_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_head_dim)},
+      {&m->attn_ws, gqa_scratch_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_kv_heads, c.fa_head_dim, c.dtype)},
       {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
       {&m->last, (size_t)B * d * es},
   };
@@ -225,7 +225,7 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
     // causal (query, key) pairs: sum over new tokens of (pos0 + t + 1)
     const double pairs = (double)B * ((double)T * pos0 + (double)T * (T + 1) / 2.0);
     const double attn_bytes = es * ((double)M * Hq * dh * 3.0 + (double)B * Hkv * (pos0 + T) * dh * 2.0);
-    CK(prof(m, s, P_ATTN, gqa_launches(B, T, pos0 + T, Hkv, m->attn_ws.p != nullptr), 4.0 * Hq * dh * pairs, attn_bytes,
+    CK(prof(m, s, P_ATTN, gqa_launches(B, T, pos0 + T, Hq, Hkv, dh, dt, m->attn_ws.p != nullptr), 4.0 * Hq * dh * pairs, attn_bytes,
             [&] { return lk::gqa_attn(m->gq.p, Hq * dh, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B, T,
                                       pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s); }),
        "GQA attention");
@@ -266,11 +266,25 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
     CK(prof(m, s, P_FA_PREP, 1, 0, 8.0 * T * (cf.rotary_dims / 2),
             [&] { return rope_table((float2*)m->rope.p, T, pos0, cf.rotary_dims, cf.rope_base, s); }),
        "rotary table");
+  // the hidden state after execution e, if e is tapped: a copy of h outside the loop block,
+  // the mean of the two streams after e's mix inside it
+  auto tap_of = [&](int e) -> void* {
+    for (size_t k = 0; k < m->tap_exec.size(); ++k)
+      if (m->tap_exec[k] == e) return m->tap_out[k];
+    return nullptr;
+  };
+  auto copy_tap = [&](void* dst) -> cudaError_t {
+    return prof(m, s, P_COPY, 1, 0, 2.0 * M * cf.d * m->esize, [&] {
+      return cudaMemcpyAsync(dst, m->h.p, M * cf.d * m->esize, cudaMemcpyDeviceToDevice, s);
+    });
+  };
   for (size_t i = 0; i < m->sched.size(); ++i) {
     const ExecRow& r = m->sched[i];
+    void* tap = tap_of(r.exec);
     if (!r.in_loop) {
       loop_status st = run_layer(m, c, r, m->h.p, m->h.p, B, T, pos0, s);
       if (st != LOOP_OK) return st;
+      if (tap) CK(copy_tap(tap), "hidden-state tap copy");
       continue;
     }
     const loop_layer_weights& w = m->layers[r.layer];
@@ -288,7 +302,13 @@ static loop_status run_stack(loop_model* m, loop_cache* c, int B, int T, cudaStr
               [&] { return mhc(MHC_MERGE, m->X.p, m->F.p, (float*)m->coeffs.p, nullptr, nullptr, nullptr, nullptr,
                                m->h.p, nullptr, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
          "mHC merge");
+      if (tap) CK(copy_tap(tap), "hidden-state tap copy");
     } else {
+      if (tap)
+        CK(prof(m, s, P_MHC, 1, 0, tok * (es * 4.0 * cf.d + 32.0),
+                [&] { return mhc(MHC_MERGE, m->X.p, m->F.p, (float*)m->coeffs.p, nullptr, nullptr, nullptr, nullptr,
+                                 tap, nullptr, (int)M, cf.d, cf.eps, cf.sinkhorn_iters, dt, s); }),
+           "hidden-state tap (stream mean)");
       const loop_layer_weights& wn = m->layers[m->sched[i + 1].layer];
       // read X (2d) + F (d), write X' (2d) + x_in (d), coefficients in/out
       CK(prof(m, s, P_MHC, 1, 0, tok * (es * 6.0 * cf.d + 64.0),
@@ -323,6 +343,9 @@ loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const 
                         float* logits_last, int B, int T, cudaStream_t s) {
   const loop_config& cf = m->cfg;
   const long M = (long)B * T;
+  if (!m->tap_exec.empty() && M > m->tap_rows)
+    return fail(LOOP_ERR_CAPACITY, "more new tokens (" + std::to_string(M) + ") than the tap buffers hold (" +
+                                       std::to_string(m->tap_rows) + " rows)");
   loop_status st = ensure_workspace(m, M, B, T, c->max_tokens, s);
   if (st != LOOP_OK) return st;
   st = prepare(m, s);
@@ -359,6 +382,9 @@ loop_status run_decode(loop_model* m, loop_cache* c, const int32_t* tok, float* 
                        cudaStream_t s) {
   const loop_config& cf = m->cfg;
   const int B = c->batch;
+  if (!m->tap_exec.empty() && B > m->tap_rows)
+    return fail(LOOP_ERR_CAPACITY, "more new tokens (" + std::to_string(B) + ") than the tap buffers hold (" +
+                                       std::to_string(m->tap_rows) + " rows)");
   loop_status st = ensure_workspace(m, B, B, 1, c->max_tokens, s);
   if (st != LOOP_OK) return st;
   st = prepare(m, s);

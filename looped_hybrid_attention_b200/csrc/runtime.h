@@ -57,6 +57,11 @@ struct loop_model {
   Profiler prof;
   DevBuf wrt;                    // [n_layers][8][2d] transposed routing maps (looped layers)
   bool wrt_ready = false;
+  // hidden-state taps (loop_set_taps): after execution tap_exec[i], the new tokens' hidden
+  // state goes to tap_out[i] [rows, d]; calls with more than tap_rows new tokens are refused
+  std::vector<int> tap_exec;
+  std::vector<void*> tap_out;
+  long tap_rows = 0;
 };
 
 struct loop_cache {
@@ -70,6 +75,12 @@ struct loop_cache {
 // Set the thread's error message; returns `st`.
 loop_status fail(loop_status st, const std::string& msg);
 loop_status cuda_fail(cudaError_t e, const char* what);
+
+// Argument checks shared by gqa_attn and gqa_attn_noalloc (same arguments, same rules).
+// Returns LOOP_OK when the call should proceed; *empty is set when it is a no-op.
+loop_status gqa_check_args(const char* who, const void* q, int ld_q, const void* k, const void* v, int kv_cap,
+                           const void* gate, int ld_gate, const void* out, int B, int Tq, int Tkv, int q_off, int Hq,
+                           int Hkv, int dh, int causal, int dtype, bool* empty);
 
 loop_status run_forward(loop_model* m, loop_cache* c, const int32_t* ids, const void* h_in, void* h_out,
                         float* logits_last, int B, int T, cudaStream_t s);

@@ -1,0 +1,235 @@
+"""Model-level parity at the stated configurations, loop passes other than two, and hidden-state taps.
+
+Each test runs the C-ABI model (loop_forward_hidden / loop_prefill / loop_decode_step)
+on seeded inputs and compares with the oracle's whole-model forward:
+  - one full-width group (3 GDN + 1 GQA, mHC around all four) at sequence length 4096, bf16;
+  - the same group at batch 64: a prefill, then three single-token steps, which run the
+    decode kernels (few-row projections, recurrent GDN step, flash-decode, mHC over a
+    64-token batch); three of the 64 sequences are checked against the oracle;
+  - the full 9B-shape stack (56 executions, "Loop-9B engineering teardown" §二) on a short
+    prefill and one decode step, with the hidden-state taps at [3, 27, 51, 53, 54]
+    ("原地套圈" investigation §03);
+  - the tiny stack with 1 and 3 loop passes (4 + 24P + 4 executions at full size, teardown
+    §六/§八), with per-execution cache slots.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import TOL, rel_l2, to64
+from oracle import model as omodel
+from oracle import ops
+from oracle import schedule as osched
+
+pytestmark = pytest.mark.gpu
+
+TINY_LM = synth.TINY.with_(with_embedding=True, vocab=1000)
+
+
+def dev_weights(w):
+    return {k: v.cuda() for k, v in w.items()}
+
+
+# ----------------------------------------------------------------------------- taps
+
+def test_tiny_taps_prefill_and_decode(cuda):
+    """Taps after executions 3, 5, 7, 11, 13, 14 of the 16-execution tiny stack (the analogues of
+    the probe points: end of the head, inside and at the end of each loop pass, the tail)."""
+    import looped_hybrid_attention_b200 as L
+    s = TINY_LM
+    w = synth.make_weights(s, seed=12)
+    W = omodel.Weights(w)
+    B, T = 2, 37
+    ids = synth.uniform_ids((B, T + 1), s.vocab, 12)
+    taps_at = [3, 5, 7, 11, 13, 14]
+    m = L.Model(s, dev_weights(w))
+    c = m.cache(B, 48)
+    bufs = [torch.full((B * T, s.d), float("nan"), device=cuda) for _ in taps_at]
+    m.set_taps(taps_at, bufs, B * T)
+    lg = torch.empty((B, s.vocab), device=cuda)
+    m.prefill(c, ids[:, :T].contiguous().cuda(), lg)
+    torch.cuda.synchronize()
+    caches = [omodel.new_cache() for _ in range(B)]
+    ref_taps = []
+    for b in range(B):
+        tb = []
+        omodel.run_stack(s, W, W["embed"][ids[b, :T].numpy()], caches[b], tb)
+        ref_taps.append(tb)
+    for i, e in enumerate(taps_at):
+        got = to64(bufs[i]).reshape(B, T, s.d)
+        for b in range(B):
+            assert rel_l2(got[b], ref_taps[b][e]) < TOL["fp32"], (e, b)
+    # decode step: B new rows per tap
+    nxt = torch.empty(B, dtype=torch.int32, device=cuda)
+    tok = ids[:, T].contiguous()
+    m.decode_step(c, tok.cuda(), lg, nxt)
+    torch.cuda.synchronize()
+    for b in range(B):
+        tb = []
+        omodel.run_stack(s, W, W["embed"][tok[b:b + 1].numpy()], caches[b], tb)
+        for i, e in enumerate(taps_at):
+            assert rel_l2(to64(bufs[i][b]), tb[e][0]) < TOL["fp32"], (e, b)
+    # a call with more new tokens than the buffers hold is refused before it launches anything
+    c2 = m.cache(B, 64)
+    with pytest.raises(L.LoopError) as err:
+        m.prefill(c2, ids[:, :T + 1].contiguous().cuda(), lg)
+    assert err.value.status == 5 and c2.length == 0
+    with pytest.raises(L.LoopError) as err:
+        m.set_taps([16], bufs[:1], B * T)                  # 16 executions: indices 0..15
+    assert err.value.status == 1
+    m.set_taps([], [], 0)                                  # cleared: the same call now runs
+    m.prefill(c2, ids[:, :T + 1].contiguous().cuda(), lg)
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------------------------- loop passes
+
+@pytest.mark.parametrize("P", [1, 3])
+def test_tiny_loop_passes_vs_oracle(cuda, P):
+    """4 + 4P + 4 executions of the tiny stack: output at 1e-5, every GDN state slot and the
+    KV slab of every FA execution equal to the oracle's cache of that execution."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.TINY.with_(loop_passes=P)
+    n_exec, n_fa, n_gdn = osched.counts(s)
+    assert n_exec == 4 + 4 * P + 4
+    assert [tuple(r) for r in L.schedule(s)] == [(e, l, int(k == "fa"), sl, int(il))
+                                                  for e, l, k, sl, il in osched.table(s)]
+    w = synth.make_weights(s, seed=20 + P)
+    T = 90
+    h = synth.normal((1, T, s.d), 1.0, 20 + P, "hidden")
+    ref, caches = omodel.forward_hidden(s, omodel.Weights(w), h)
+    m = L.Model(s, dev_weights(w))
+    c = m.cache(1, 96)
+    out = torch.empty((1, T, s.d), device=cuda)
+    m.forward_hidden(c, h.cuda(), out)
+    torch.cuda.synchronize()
+    assert rel_l2(to64(out), ref) < TOL["fp32"]
+    for slot in range(n_gdn):
+        st = L.device_view(c.state_ptr(slot), (1, s.gdn_heads, s.gdn_dv, s.gdn_dk), torch.float32)
+        assert rel_l2(to64(st[0]), caches[0]["state"][slot]) < 1e-4, slot
+    errs = np.zeros((n_fa, n_fa))
+    for slot in range(n_fa):
+        K = L.device_view(c.kv_ptrs(slot)[0], (1, s.fa_kv_heads, 96, s.fa_head_dim), torch.float32)
+        got = to64(K[0, :, :T]).transpose(1, 0, 2)
+        for o in range(n_fa):
+            errs[slot, o] = rel_l2(got, caches[0]["kv"][o][0])
+    assert np.all(np.diag(errs) < 1e-5)
+    assert np.all(errs[~np.eye(n_fa, dtype=bool)] > 1e-2)
+
+
+# ----------------------------------------------------------------------------- full-width group
+
+@pytest.mark.slow
+def test_group_bf16_seq4096_vs_oracle(cuda):
+    """The one-group configuration as stated: batch 1, sequence 4096, bf16 weights N(0, 0.02),
+    inputs N(0, 1); the output hidden states within the bf16 end-to-end tolerance."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.GROUP
+    T = 4096
+    w = synth.make_weights(s, seed=2)
+    h = synth.normal((1, T, s.d), 1.0, 2, "hidden").to(torch.bfloat16)
+    m = L.Model(s, dev_weights(w))
+    c = m.cache(1, T)
+    out = torch.empty((1, T, s.d), dtype=torch.bfloat16, device=cuda)
+    m.forward_hidden(c, h.cuda(), out)
+    torch.cuda.synchronize()
+    ref, _ = omodel.forward_hidden(s, omodel.Weights(w), h)
+    got = to64(out)
+    assert rel_l2(got, ref) < TOL["bf16_e2e"]
+    assert rel_l2(got[0, -512:], ref[0, -512:]) < TOL["bf16_e2e"]      # the late rows on their own
+
+
+@pytest.mark.slow
+def test_group_bf16_batch64_prefill_then_decode(cuda):
+    """Batch 64: a 64-token prefill, then three single-token forwards (the decode kernels);
+    sequences 0, 29 and 63 against the oracle after every call."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.GROUP
+    B, T0, steps = 64, 64, 3
+    w = synth.make_weights(s, seed=6)
+    W = omodel.Weights(w)
+    h = synth.normal((B, T0 + steps, s.d), 1.0, 6, "hidden").to(torch.bfloat16)
+    m = L.Model(s, dev_weights(w))
+    c = m.cache(B, T0 + steps)
+    hd = h.cuda()
+    out = torch.empty((B, T0, s.d), dtype=torch.bfloat16, device=cuda)
+    m.forward_hidden(c, hd[:, :T0].contiguous(), out)
+    outs = []
+    for t in range(steps):
+        o = torch.empty((B, 1, s.d), dtype=torch.bfloat16, device=cuda)
+        m.forward_hidden(c, hd[:, T0 + t:T0 + t + 1].contiguous(), o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0 and c.length == T0 + steps
+    for b in (0, 29, 63):
+        cache = omodel.new_cache()
+        ref = omodel.run_stack(s, W, h[b, :T0], cache)
+        assert rel_l2(to64(out[b]), ref) < TOL["bf16_e2e"], b
+        for t in range(steps):
+            ref = omodel.run_stack(s, W, h[b, T0 + t:T0 + t + 1], cache)
+            assert rel_l2(to64(outs[t][b]), ref) < TOL["bf16_e2e"], (b, t)
+
+
+# ----------------------------------------------------------------------------- full 9B-shape stack
+
+class _RowGather:
+    """Rows of a device embedding table, widened on demand."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, idx):
+        return ops.f64(self.t[torch.as_tensor(np.asarray(idx), device=self.t.device)])
+
+
+class _StreamedWeights(omodel.Weights):
+    """Widens each tensor on every access instead of keeping it: the full stack in float64
+    would take 65 GB of host memory, one layer at a time takes under 2 GB."""
+
+    def __getitem__(self, name):
+        if name == "embed":
+            return _RowGather(self._t[name])
+        return ops.f64(self._t[name])
+
+
+@pytest.mark.slow
+def test_full_stack_prefill_decode_and_taps_vs_oracle(cuda):
+    """The 9B-shape stack (32 stored layers, 56 executions, bf16, random init) at batch 1:
+    a 40-token prefill and one greedy decode step against the oracle, with the hidden-state
+    taps at executions [3, 27, 51, 53, 54]."""
+    import looped_hybrid_attention_b200 as L
+    s = synth.FULL
+    T = 40
+    taps_at = [3, 27, 51, 53, 54]
+    w = synth.make_weights(s, seed=0, device=cuda)
+    ids = synth.uniform_ids((1, T + 1), s.vocab, 31)
+    m = L.Model(s, w)
+    c = m.cache(1, 64)
+    bufs = [torch.empty((T, s.d), dtype=torch.bfloat16, device=cuda) for _ in taps_at]
+    m.set_taps(taps_at, bufs, T)
+    lg = torch.empty((1, s.vocab), device=cuda)
+    m.prefill(c, ids[:, :T].contiguous().cuda(), lg)
+    torch.cuda.synchronize()
+    got_taps = [to64(b) for b in bufs]
+    got_lg = to64(lg)
+    nxt = torch.empty(1, dtype=torch.int32, device=cuda)
+    lg2 = torch.empty_like(lg)
+    m.decode_step(c, ids[:, T].contiguous().cuda(), lg2, nxt)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+
+    W = _StreamedWeights(w)
+    cache = omodel.new_cache()
+    taps = []
+    hT = omodel.run_stack(s, W, W["embed"][ids[0, :T].numpy()], cache, taps)
+    assert len(taps) == 56
+    ref_lg = ops.lm_logits(hT[-1:], W["final_norm"], W["lm_head"], s.eps)
+    assert rel_l2(got_lg, ref_lg) < TOL["bf16_e2e"]
+    for i, e in enumerate(taps_at):
+        assert rel_l2(got_taps[i], taps[e]) < TOL["bf16_e2e"], e
+    ref_lg2, ref_next = omodel.decode_step(s, W, [cache], ids[:, T].numpy())
+    assert rel_l2(to64(lg2), ref_lg2) < TOL["bf16_e2e"]
+    srt = np.sort(ref_lg2[0])
+    if srt[-1] - srt[-2] > 1e-2 * abs(srt[-1]):
+        assert int(nxt[0]) == int(ref_next[0])

@@ -55,7 +55,7 @@ def test_mhc_modes(cuda, dtype, d, N):
     pre, post, res = ops.mhc_coeffs(Xo, to64(w_r), to64(b_r), eps, iters)
     c = to64(c0)
     assert rel_l2(c[:, 0:2], pre) < 1e-5 and rel_l2(c[:, 2:4], post) < 1e-5
-    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() < 1e-5
+    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() <= TOL["sinkhorn"]
     assert rel_l2(to64(x_in), ops.mhc_read(Xo, c[:, 0:2])) < tol
     # MIX: X' = H_res X + H_post F, then route from X' as stored
     X_prev = X.clone()
@@ -66,7 +66,7 @@ def test_mhc_modes(cuda, dtype, d, N):
     pre, post, res = ops.mhc_coeffs(to64(X), to64(w_r), to64(b_r), eps, iters)
     c = to64(c1)
     assert rel_l2(c[:, 0:2], pre) < 1e-5 and rel_l2(c[:, 2:4], post) < 1e-5
-    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() < 1e-5
+    assert np.abs(c[:, 4:8].reshape(N, 2, 2) - res).max() <= TOL["sinkhorn"]
     assert rel_l2(to64(x_in), ops.mhc_read(to64(X), pre)) < tol
     # ROUTE only: X unchanged
     X_keep = X.clone()
@@ -95,6 +95,50 @@ def test_mhc_zero_routing_is_plain_residual(cuda):
     hm = torch.empty_like(h)
     L.mhc_route_mix(L.MHC_MERGE, X, F, c, None, None, None, None, hm, None, N, d, 1e-6, 20, L.F32)
     assert torch.allclose(hm, h + F, atol=1e-5)
+
+
+def _residual_logit_sets():
+    """2x2 residual logits with spreads (max - min) from 0.1 to 100: both sides of the 40 at which
+    the fused kernel's Sinkhorn changes from the row-odds recurrence to literal divisions."""
+    r = np.random.default_rng(17)
+    sets = []
+    for spread in (0.1, 1.0, 4.0, 10.0, 25.0, 39.5, 40.5, 60.0, 100.0):
+        for _ in range(3):
+            l = r.uniform(0.0, 1.0, size=4)
+            l = (l - l.min()) / (l.max() - l.min()) * spread - spread / 2
+            sets.append(l)
+    return sets
+
+
+@pytest.mark.parametrize("dtype,d,N", [("fp32", 256, 10), ("fp32", 256, 1100), ("bf16", 4096, 10),
+                                       ("bf16", 4096, 64), ("bf16", 4096, 1100)])
+def test_mhc_sinkhorn_of_bias_only_routing(cuda, dtype, d, N):
+    """With w_r = 0 the routing logits are exactly b_r for every token, so the fused kernel's
+    H_res is the 20-iteration Sinkhorn of exp(b_r[4:8]) and must match it within 1e-6 (FP32
+    Sinkhorn, "Loop-9B engineering teardown" §五), in the routing of OPEN and of MIX."""
+    import looped_hybrid_attention_b200 as L
+    code = L.BF16 if dtype == "bf16" else L.F32
+    h = rnd((N, d), 31, "hs", dtype=dtype)
+    F = rnd((N, d), 32, "Fs", dtype=dtype)
+    w_r = torch.zeros((2 * d, 8), device=cuda)
+    X = torch.empty((N, 2, d), dtype=DT[dtype], device=cuda)
+    x_in = torch.empty((N, d), dtype=DT[dtype], device=cuda)
+    c0, c1 = torch.empty((N, 8), device=cuda), torch.empty((N, 8), device=cuda)
+    worst = 0.0
+    for l4 in _residual_logit_sets():
+        b = np.concatenate([np.array([0.3, -1.2, 0.8, 2.5]), l4]).astype(np.float32)
+        b_r = torch.tensor(b, device=cuda)
+        ref = ops.sinkhorn(b[4:8].astype(np.float64).reshape(2, 2), 20)
+        L.mhc_route_mix(L.MHC_OPEN, h, None, None, w_r, b_r, X, x_in, None, c0, N, d, 1e-6, 20, code)
+        L.mhc_route_mix(L.MHC_MIX, X, F, c0, w_r, b_r, X, x_in, None, c1, N, d, 1e-6, 20, code)
+        for c in (to64(c0), to64(c1)):
+            assert np.isfinite(c).all()
+            err = np.abs(c[:, 4:8].reshape(N, 2, 2) - ref[None]).max()
+            worst = max(worst, err)
+            assert err <= TOL["sinkhorn"], (l4, err)
+            assert np.abs(c[:, 0:2] - ops.sigmoid(b[0:2].astype(np.float64))).max() < 1e-6
+            assert np.abs(c[:, 2:4] - 2 * ops.sigmoid(b[2:4].astype(np.float64))).max() < 2e-6
+    assert worst <= TOL["sinkhorn"]
 
 
 @pytest.mark.parametrize("N", [10, 1100])
