@@ -45,7 +45,17 @@ def layer_branch(shape, W, l, kind, slot, x, cache, pos0):
     s = shape
     lw = W.layer(l)
     a = ops.rmsnorm(x, lw("attn_norm"), s.eps)
-    if kind == "gdn":
+    if kind == "gdn" and getattr(s, "gdn_variant", 0) == 1:
+        Hk, Hv, dk, dv = s.gdn_heads, s.gdn_v_heads or s.gdn_heads, s.gdn_dk, s.gdn_dv
+        S0 = cache["state"].get(slot)
+        if S0 is None:
+            S0 = np.zeros((Hv, dv, dk))                # READING: zero state and conv inputs at sequence start
+        conv0 = cache.setdefault("conv", {}).get(slot)
+        mix, S, conv = ops.gdn_mixer_v2(a, lw("gdn_w_in"), lw("gdn_conv_w"), lw("gdn_a_bias"), lw("gdn_b_bias"),
+                                        lw("gdn_o_norm"), lw("gdn_w_out"), S0, conv0, Hk, Hv, dk, dv, s.eps)
+        cache["state"][slot] = S
+        cache["conv"][slot] = conv
+    elif kind == "gdn":
         H, dk, dv = s.gdn_heads, s.gdn_dk, s.gdn_dv
         S0 = cache["state"].get(slot)
         if S0 is None:

@@ -132,6 +132,75 @@ def gdn_mixer(x_normed, w_in, a_bias, b_bias, w_out, S0, H, dk, dv, eps):
     return linear(o.reshape(o.shape[0], H * dv), w_out), S
 
 
+# ----------------------------------------------------------------------------- GDN variant: short conv + gated output norm
+
+def causal_conv_silu(x, w, state):
+    """Depthwise causal convolution over time, then SiLU, per channel.
+
+    READING ([probe] §01 names the backbone qwen3_5_text; its Gated-DeltaNet layers pass
+    the q, k, v channels through a short causal depthwise convolution and SiLU before the
+    recurrence): x [T, C]; w [C, K]; state [K-1, C] = the K-1 inputs before x (zeros at
+    sequence start).  y_t[c] = silu(sum_j w[c, j] * x_{t-(K-1)+j}[c]), so w[:, K-1] weighs
+    the current token.  Returns y [T, C] and the new state (the last K-1 inputs).
+    """
+    x, w = f64(x), f64(w)
+    K = w.shape[1]
+    st = np.zeros((K - 1, x.shape[1])) if state is None else f64(state)
+    ext = np.concatenate([st, x], axis=0)                      # [K-1+T, C]
+    T = x.shape[0]
+    y = np.zeros_like(x)
+    for t in range(T):
+        for j in range(K):
+            y[t] += w[:, j] * ext[t + j]
+    return silu(y), ext[T:].copy()
+
+
+def gated_rmsnorm(o, z, w, eps):
+    """Output gate of the variant: RMSNorm of each head's output (gain w over dv) times silu(z).
+
+    o, z [T, H, dv] -> [T, H, dv].  READING: the gated output norm of the qwen3_5_text
+    Gated-DeltaNet layer ([probe] §01).
+    """
+    return rmsnorm(o, w, eps) * silu(f64(z))
+
+
+def gdn_split_projection_v2(P, Hk, Hv, dk, dv):
+    """Split the variant's input projection into q, k (Hk heads), v, z (Hv heads), a, b (Hv)."""
+    T = P.shape[0]
+    o = 0
+    q = P[:, o:o + Hk * dk]; o += Hk * dk
+    k = P[:, o:o + Hk * dk]; o += Hk * dk
+    v = P[:, o:o + Hv * dv]; o += Hv * dv
+    z = P[:, o:o + Hv * dv].reshape(T, Hv, dv); o += Hv * dv
+    a = P[:, o:o + Hv]; o += Hv
+    b = P[:, o:o + Hv]
+    return q, k, v, z, a, b
+
+
+def gdn_mixer_v2(x_normed, w_in, conv_w, a_bias, b_bias, o_norm, w_out, S0, conv0, Hk, Hv, dk, dv, eps):
+    """GDN token mixer of the variant ([probe] §01: backbone qwen3_5_text).
+
+    READING: projections q, k (Hk heads), v, z (Hv heads), a, b (Hv); the q | k | v
+    channels pass through causal_conv_silu; q and k are L2-normalised per head; value
+    head h reads key head h // (Hv // Hk); gates and recurrence as in gdn_mixer; each
+    head's output goes through gated_rmsnorm with z; then the output map.
+    Returns (mix, final state [Hv, dv, dk], conv state [K-1, 2*Hk*dk + Hv*dv]).
+    """
+    P = linear(x_normed, w_in)
+    T = P.shape[0]
+    q, k, v, z, a, b = gdn_split_projection_v2(P, Hk, Hv, dk, dv)
+    y, conv_new = causal_conv_silu(np.concatenate([q, k, v], axis=1), conv_w, conv0)
+    q = l2norm(y[:, :Hk * dk].reshape(T, Hk, dk), eps)
+    k = l2norm(y[:, Hk * dk:2 * Hk * dk].reshape(T, Hk, dk), eps)
+    v = y[:, 2 * Hk * dk:].reshape(T, Hv, dv)
+    rep = Hv // Hk
+    q, k = np.repeat(q, rep, axis=1), np.repeat(k, rep, axis=1)     # head h -> key head h // rep
+    g, beta = gdn_gates(a, b, a_bias, b_bias)
+    o, S = gdn_recurrent(q, k, v, g, beta, S0, 1.0 / np.sqrt(dk))
+    o = gated_rmsnorm(o, z, o_norm, eps)
+    return linear(o.reshape(T, Hv * dv), w_out), S, conv_new
+
+
 # ----------------------------------------------------------------------------- full attention
 
 def rope(x, pos, rotary_dims, base):

@@ -50,6 +50,9 @@ class ModelShape:
     rope_base: float = 10000.0
     dtype: str = "bf16"           # storage dtype of weights and activations
     with_embedding: bool = True   # False: hidden-state in/out (tiny and group configs)
+    gdn_variant: int = 0          # 0: plain GDN; 1: short causal conv on q|k|v + gated output norm
+    gdn_v_heads: int = 0          # value heads of the variant (0: gdn_heads); a multiple of gdn_heads
+    gdn_conv: int = 4             # conv kernel size of the variant
 
     def as_dict(self):
         return asdict(self)
@@ -112,7 +115,9 @@ def weight_names(shape: ModelShape):
     """Names and shapes of every tensor of the model, in a fixed order.
 
     Row-major, nn.Linear convention: a projection weight is [out, in].
-    GDN input projection rows: q (H*dk) | k (H*dk) | v (H*dv) | a (H) | b (H).
+    GDN input projection rows: q (H*dk) | k (H*dk) | v (H*dv) | a (H) | b (H); for the
+    variant (gdn_variant 1): q, k (Hk = gdn_heads) | v, z (Hv = gdn_v_heads) | a, b (Hv),
+    conv weights [2*Hk*dk + Hv*dv, gdn_conv] and an output-norm gain [dv].
     FA input projection rows:  q (Hq*dh) | gate (Hq*dh) | k (Hkv*dh) | v (Hkv*dh).
     mHC routing map w_r is [streams*d, 8] fp32; b_r is [8] fp32.
     """
@@ -123,7 +128,15 @@ def weight_names(shape: ModelShape):
     for l, kind in enumerate(layer_kinds(s)):
         p = f"layers.{l}."
         out.append((p + "attn_norm", (s.d,), "gain"))
-        if kind == "gdn":
+        if kind == "gdn" and s.gdn_variant == 1:
+            Hk, Hv, dk, dv = s.gdn_heads, s.gdn_v_heads or s.gdn_heads, s.gdn_dk, s.gdn_dv
+            out.append((p + "gdn_w_in", (2 * Hk * dk + 2 * Hv * dv + 2 * Hv, s.d), "store"))
+            out.append((p + "gdn_conv_w", (2 * Hk * dk + Hv * dv, s.gdn_conv), "store"))
+            out.append((p + "gdn_a_bias", (Hv,), "fp32"))
+            out.append((p + "gdn_b_bias", (Hv,), "fp32"))
+            out.append((p + "gdn_o_norm", (dv,), "gain"))
+            out.append((p + "gdn_w_out", (s.d, Hv * dv), "store"))
+        elif kind == "gdn":
             H, dk, dv = s.gdn_heads, s.gdn_dk, s.gdn_dv
             out.append((p + "gdn_w_in", (2 * H * dk + H * dv + 2 * H, s.d), "store"))
             out.append((p + "gdn_a_bias", (H,), "fp32"))
