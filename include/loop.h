@@ -73,6 +73,11 @@ typedef struct loop_config {
   float eps, rope_base;
   int dtype;             /* loop_dtype */
   int with_embedding;    /* 1: token ids in, logits out; 0: hidden states in/out */
+  /* GDN variant ("原地套圈" investigation §01 declares the backbone qwen3_5_text):
+   * 0 = plain GDN; 1 = causal depthwise conv (gdn_conv taps) + SiLU on the q | k | v
+   * channels and a gated RMSNorm of each head's output, with gdn_v_heads value heads
+   * (0 = gdn_heads; a multiple of gdn_heads) reading gdn_heads key heads. */
+  int gdn_variant, gdn_v_heads, gdn_conv;
 } loop_config;
 
 /* Weights of one stored layer; device pointers, caller-owned, must outlive the model.
@@ -81,6 +86,7 @@ typedef struct loop_config {
 typedef struct loop_layer_weights {
   const void* attn_norm;      /* [d] pre-mixer RMSNorm gain */
   const void* w_in;           /* GDN: [2*H*dk + H*dv + 2*H, d], row blocks q | k | v | a | b
+                                 GDN variant: [2*Hk*dk + 2*Hv*dv + 2*Hv, d], q | k | v | z | a | b
                                  FA:  [2*Hq*dh + 2*Hkv*dh, d],  row blocks q | gate | k | v */
   const float* gdn_a_bias;    /* GDN [H] fp32: decay gate g = -softplus(a + a_bias) */
   const float* gdn_b_bias;    /* GDN [H] fp32: beta = sigmoid(b + b_bias) */
@@ -93,6 +99,8 @@ typedef struct loop_layer_weights {
   const void* w_down;         /* [d, ffn] */
   const float* mhc_w_r;       /* looped layers: [streams*d, 8] fp32 routing map, else NULL */
   const float* mhc_b_r;       /* looped layers: [8] fp32 routing bias, else NULL */
+  const void* gdn_conv_w;     /* GDN variant: [2*Hk*dk + Hv*dv, gdn_conv] conv taps (last = current token) */
+  const void* gdn_o_norm;     /* GDN variant: [dv] gain of the gated output norm */
 } loop_layer_weights;
 
 typedef struct loop_weights {
@@ -131,7 +139,10 @@ loop_status loop_model_destroy(loop_model* m);
  * Owns n_fa KV slabs, each K and V [batch, Hkv, max_tokens, dh] (dtype), and n_gdn
  * GDN states [batch, H, dv, dk] fp32 ("Loop-9B engineering teardown" §四: the two
  * loop passes keep separate caches).  Bytes = n_fa*2*batch*Hkv*max_tokens*dh*esize
- * + n_gdn*batch*H*dv*dk*4.  New caches are zero with length 0. */
+ * + n_gdn*batch*H*dv*dk*4.  The GDN variant's states have H = Hv value heads, and each
+ * GDN execution also keeps its last gdn_conv - 1 conv inputs [batch, gdn_conv-1, C]
+ * (dtype, C = 2*Hk*dk + Hv*dv), counted in state_bytes.  New caches are zero with
+ * length 0. */
 loop_status loop_cache_create(const loop_model* m, int batch, int max_tokens, loop_cache** out);
 loop_status loop_cache_reset(loop_cache* c);          /* length 0, states zeroed (on the default stream) */
 loop_status loop_cache_destroy(loop_cache* c);
@@ -197,6 +208,26 @@ loop_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
                           void* stream);
 size_t loop_gdn_workspace_bytes(int B, int T, int H, int dk, int dv);
 
+/* GDN variant input preparation ("原地套圈" investigation §01, backbone qwen3_5_text): from
+ * P [B*T, ld_p] (row blocks q | k (Hk heads) | v | z (Hv heads) | a | b (Hv)): the q | k | v
+ * channels c pass through a causal depthwise conv and SiLU,
+ *   y_t[c] = silu(sum_{j<conv} conv_w[c][j] * x_{t-(conv-1)+j}[c]),
+ * where inputs before the call's first token come from conv_state [B, conv-1, C] (dtype,
+ * in/out: afterwards it holds the last conv-1 inputs); then q, k are L2-normalised per head
+ * (x / sqrt(sum x^2 + eps)) and written once per value head h that reads key head
+ * h / (Hv/Hk): q, k [B*T, Hv, dk]; v [B*T, Hv, dv]; g = -softplus(a + a_bias),
+ * beta = sigmoid(b + b_bias) [B*T, Hv] fp32.  conv must be 4; (dk, dv) as gdn_chunk_fwd. */
+loop_status gdn_conv_prep(const void* P, int ld_p, const void* conv_w, void* conv_state,
+                          const float* a_bias, const float* b_bias, void* q, void* k, void* v,
+                          float* g, float* beta, int B, int T, int Hk, int Hv, int dk, int dv,
+                          int conv, float eps, int dtype, void* stream);
+
+/* Gated output norm of the GDN variant: y [M, H, dv] = RMSNorm(o) * w * silu(z) per head
+ * (RMSNorm over dv with eps inside the root); o [M, H, dv], z rows of stride ld_z
+ * elements ([M, H*dv] blocks), w [dv]; y may equal o.  dv a multiple of 32, <= 256. */
+loop_status gdn_gated_norm(const void* o, const void* z, int ld_z, const void* w, void* y, int M, int H,
+                           int dv, float eps, int dtype, void* stream);
+
 /* One token of the same recurrence per sequence: q, k [B, H, dk]; v, out [B, H, dv];
  * g, beta [B, H] fp32; state [B, H, dv, dk] fp32 in/out. */
 loop_status gdn_step(const void* q, const void* k, const void* v, const float* g,
@@ -253,11 +284,26 @@ loop_status gqa_attn_noalloc(const void* q, int ld_q, const void* k, const void*
                              const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv,
                              int q_off, int Hq, int Hkv, int dh, int causal, int dtype, void* stream);
 
+/* gqa_attn with the query side of "Loop-9B engineering teardown" §三 fused in: q are the
+ * raw query rows of the input projection (row stride ld_q), and the kernel applies
+ * QK-norm and rotary to them as it loads them, q' = rope(rmsnorm(q) * q_norm) (RMSNorm
+ * over the dh dims with eps inside the root; dims [0, rotary_dims) rotated in adjacent
+ * pairs (2j, 2j+1) by angle pos * rope_base^(-2j/rotary_dims), pos = q_off + t).  k and v
+ * are the slab as fa_prep writes it (keys already normed and rotated).  Built for the
+ * tensor-core kernel only: bf16, dh 256, Tq >= 16, 128 % (Hq/Hkv) == 0, rotary_dims <=
+ * dh/2, 16-byte aligned q, q_norm, k, v, gate; other calls return LOOP_ERR_UNSUPPORTED.
+ * Needs no workspace. */
+loop_status gqa_attn_fused_q(const void* q, int ld_q, const void* q_norm, int rotary_dims, float rope_base,
+                             float eps, const void* k, const void* v, int kv_cap, const void* gate,
+                             int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv,
+                             int dh, int causal, int dtype, void* stream);
+
 /* QK-norm + partial rotary + KV write for one FA execution.  From P [M = B*T, ld_p]
  * (row blocks q | gate | k | v): q_out [M, Hq, dh] = rope(rmsnorm(q) * q_norm);
  * k = rope(rmsnorm(k) * k_norm) and v are written to the slabs k_cache, v_cache
  * [B, Hkv, kv_cap, dh] at positions pos0 .. pos0+T-1.  Rotary: dims [0, rotary_dims)
- * in adjacent pairs (2j, 2j+1), angle = pos * base^(-2j/rotary_dims). */
+ * in adjacent pairs (2j, 2j+1), angle = pos * base^(-2j/rotary_dims).  q_out may be NULL:
+ * then only the keys and values are written (the queries go raw to gqa_attn_fused_q). */
 loop_status fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm,
                     void* q_out, void* k_cache, void* v_cache, int kv_cap, int B, int T, int pos0,
                     int Hq, int Hkv, int dh, int rotary_dims, float rope_base, float eps,

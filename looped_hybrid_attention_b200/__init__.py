@@ -39,13 +39,14 @@ class loop_config(ctypes.Structure):
         "gdn_heads", "gdn_dk", "gdn_dv", "fa_q_heads", "fa_kv_heads", "fa_head_dim", "rotary_dims",
         "mhc_streams", "sinkhorn_iters", "gdn_chunk")] + [
         ("eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("dtype", ctypes.c_int),
-        ("with_embedding", ctypes.c_int)]
+        ("with_embedding", ctypes.c_int), ("gdn_variant", ctypes.c_int), ("gdn_v_heads", ctypes.c_int),
+        ("gdn_conv", ctypes.c_int)]
 
 
 class loop_layer_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "attn_norm", "w_in", "gdn_a_bias", "gdn_b_bias", "q_norm", "k_norm", "w_out", "ffn_norm",
-        "w_gate", "w_up", "w_down", "mhc_w_r", "mhc_b_r")]
+        "w_gate", "w_up", "w_down", "mhc_w_r", "mhc_b_r", "gdn_conv_w", "gdn_o_norm")]
 
 
 class loop_profile_entry(ctypes.Structure):
@@ -81,10 +82,13 @@ _SIGS = {
     "gdn_chunk_fwd": ([_P] * 7 + [_I] * 6 + [_F, _P, _I, _P], _I),
     "loop_gdn_workspace_bytes": ([_I] * 5, _Z),
     "gdn_step": ([_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
+    "gdn_conv_prep": ([_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P] + [_I] * 7 + [_F, _I, _P], _I),
+    "gdn_gated_norm": ([_P, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P], _I),
     "gdn_prep": ([_P, _I] + [_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
     "gqa_attn": ([_P, _I, _P, _P, _I, _P, _I, _P] + [_I] * 8 + [_P, _I, _P], _I),
     "loop_gqa_workspace_bytes": ([_I] * 5, _Z),
     "gqa_attn_noalloc": ([_P, _I, _P, _P, _I, _P, _I, _P] + [_I] * 8 + [_I, _P], _I),
+    "gqa_attn_fused_q": ([_P, _I, _P, _I, _F, _F, _P, _P, _I, _P, _I, _P] + [_I] * 9 + [_P], _I),
     "fa_prep": ([_P, _I, _P, _P, _P, _P, _P, _I] + [_I] * 7 + [_F, _F, _I, _P], _I),
     "mhc_route_mix": ([_I] + [_P] * 9 + [_I, _I, _F, _I, _I, _P], _I),
     "sinkhorn_fp32": ([_P, _P, _I, _I, _I, _P], _I),
@@ -163,7 +167,8 @@ def make_config(shape) -> loop_config:
     return loop_config(s.d, s.ffn, s.vocab, s.n_layers, s.loop_start, s.loop_end, s.loop_passes, s.group,
                        s.gdn_heads, s.gdn_dk, s.gdn_dv, s.fa_q_heads, s.fa_kv_heads, s.fa_head_dim,
                        s.rotary_dims, s.mhc_streams, s.sinkhorn_iters, s.gdn_chunk, s.eps, s.rope_base,
-                       BF16 if s.dtype == "bf16" else F32, 1 if s.with_embedding else 0)
+                       BF16 if s.dtype == "bf16" else F32, 1 if s.with_embedding else 0,
+                       getattr(s, "gdn_variant", 0), getattr(s, "gdn_v_heads", 0), getattr(s, "gdn_conv", 4))
 
 
 def schedule(shape):
@@ -194,7 +199,8 @@ class Model:
             layers[l] = loop_layer_weights(
                 g("attn_norm"), g("fa_w_in" if fa else "gdn_w_in"), g("gdn_a_bias"), g("gdn_b_bias"),
                 g("fa_q_norm"), g("fa_k_norm"), g("fa_w_out" if fa else "gdn_w_out"), g("ffn_norm"),
-                g("ffn_w_gate"), g("ffn_w_up"), g("ffn_w_down"), g("mhc_w_r"), g("mhc_b_r"))
+                g("ffn_w_gate"), g("ffn_w_up"), g("ffn_w_down"), g("mhc_w_r"), g("mhc_b_r"),
+                g("gdn_conv_w"), g("gdn_o_norm"))
         self._layers = layers
         w = loop_weights(ptr(weights.get("embed")), ptr(weights.get("final_norm")), ptr(weights.get("lm_head")),
                          layers, s.n_layers)
@@ -315,6 +321,19 @@ def gdn_prep(P, a_bias, b_bias, q, k, v, g, beta, H, dk, dv, eps, stream=None):
                         M, H, dk, dv, eps, dtype_code(P), _stream(stream)), "gdn_prep")
 
 
+def gdn_conv_prep(P, conv_w, conv_state, a_bias, b_bias, q, k, v, g, beta, B, T, Hk, Hv, dk, dv, eps, conv=4,
+                  stream=None):
+    """GDN variant input preparation: conv + SiLU on q|k|v, L2 norm, gates; conv_state updated in place."""
+    check(_lib.gdn_conv_prep(ptr(P), P.stride(0), ptr(conv_w), ptr(conv_state), ptr(a_bias), ptr(b_bias), ptr(q),
+                             ptr(k), ptr(v), ptr(g), ptr(beta), B, T, Hk, Hv, dk, dv, conv, eps, dtype_code(P),
+                             _stream(stream)), "gdn_conv_prep")
+
+
+def gdn_gated_norm(o, z, ld_z, w, y, M, H, dv, eps, stream=None):
+    check(_lib.gdn_gated_norm(ptr(o), ptr(z), ld_z, ptr(w), ptr(y), M, H, dv, eps, dtype_code(o), _stream(stream)),
+          "gdn_gated_norm")
+
+
 def gqa_workspace_bytes(B, Tq, Tkv, Hq, dh):
     return _lib.loop_gqa_workspace_bytes(B, Tq, Tkv, Hq, dh)
 
@@ -330,6 +349,14 @@ def gqa_attn_noalloc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_of
     """gqa_attn with the split-K scratch in the library's fixed device array (allocates nothing)."""
     check(_lib.gqa_attn_noalloc(ptr(q), ld_q, ptr(k), ptr(v), kv_cap, ptr(gate), ld_gate, ptr(out), B, Tq, Tkv,
                                 q_off, Hq, Hkv, dh, int(causal), dtype_code(q), _stream(stream)), "gqa_attn_noalloc")
+
+
+def gqa_attn_fused_q(q, ld_q, q_norm, rotary_dims, rope_base, eps, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv,
+                     q_off, Hq, Hkv, dh, causal=True, stream=None):
+    """gqa_attn on raw query rows: QK-norm and rotary applied by the attention kernel."""
+    check(_lib.gqa_attn_fused_q(ptr(q), ld_q, ptr(q_norm), rotary_dims, rope_base, eps, ptr(k), ptr(v), kv_cap,
+                                ptr(gate), ld_gate, ptr(out), B, Tq, Tkv, q_off, Hq, Hkv, dh, int(causal),
+                                dtype_code(q), _stream(stream)), "gqa_attn_fused_q")
 
 
 def fa_prep(P, q_norm, k_norm, q_out, k_cache, v_cache, kv_cap, B, T, pos0, Hq, Hkv, dh, rotary_dims, rope_base,

@@ -49,11 +49,12 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
                                                       float eps, const float2* __restrict__ tab) {
   constexpr int PER = DH / 32;         // contiguous elements per lane (even: rotary pairs stay local)
   const int lane = threadIdx.x & 31;
-  const int groups = (Hq + Hkv) / R;
+  const int hq = q_out ? Hq : 0;       // no q_out: keys and values only
+  const int groups = (hq + Hkv) / R;
   const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int b = blockIdx.y;
   if (w >= (long)T_len * groups) return;
-  const int t = (int)(w / groups), hh0 = (int)(w % groups) * R;
+  const int t = (int)(w / groups), hh0 = (int)(w % groups) * R + (Hq - hq);
   const long m = (long)b * T_len + t;
   const int pos = pos0 + t;
   const T* row = P + m * ld_p;
@@ -164,8 +165,9 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
   const int es = dtype == BF16 ? 2 : 4;
   const bool vec = al16(P) && al16(q_norm) && al16(k_norm) && al16(q_out) && al16(k_cache) && al16(v_cache) &&
                    ((long)ld_p * es) % 16 == 0;
-  const int R = (vec && Hq % 4 == 0 && Hkv % 4 == 0) ? 4 : 1;   // heads per warp
-  dim3 grid((unsigned)(((long)T * ((Hq + Hkv) / R) + warps - 1) / warps), B);
+  const int hq = q_out ? Hq : 0;                                // no q_out: keys and values only
+  const int R = (vec && hq % 4 == 0 && Hkv % 4 == 0) ? 4 : 1;   // heads per warp
+  dim3 grid((unsigned)(((long)T * ((hq + Hkv) / R) + warps - 1) / warps), B);
 #define FA_PREP(TT, DHV)                                                                                   \
   do {                                                                                                     \
     if (R == 4) FA_PREP_V(TT, DHV, true, 4);                                                               \
@@ -798,10 +800,17 @@ static cudaError_t launch_attn(const void* q, int ld_q, const void* k, const voi
 cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
                      const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
-                     cudaStream_t s) {
+                     cudaStream_t s, const QNorm* qn) {
   if (B == 0 || Tq == 0) return cudaSuccess;
   auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
   const AttnPath path = attn_path(Tq, dtype, dh, Hq, Hkv);
+  // raw queries (normalised and rotated while staged) only on the tensor-core kernel
+  if (qn) {
+    if (path != ATT_TC || !al16(qn->gain)) return cudaErrorNotSupported;
+    if (Tkv == 0) return cudaSuccess;
+    if (!gqa_tc_supported(dh, dtype, q, ld_q, gate, ld_gate, k, v, kv_cap)) return cudaErrorNotSupported;
+    return gqa_attn_tc(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, causal, s, qn);
+  }
   // The tiled kernels move 16-byte pieces (TMA boxes, cp.async); a call whose shape selects one of
   // them but whose buffers are not 16-byte aligned is refused rather than run on a slower kernel.
   if (path == ATT_TC) {

@@ -21,6 +21,11 @@
 //         the running max grows by more than 2^8 (the stale max cancels in the final
 //         O / l); finally O / l * sigmoid(gate) is stored.  Each thread first writes
 //         its half of its row of Q into shared memory (128-byte swizzled quarters).
+//         With a query-norm gain the rows are read raw from the input projection and
+//         normalised and rotated on the way ("Loop-9B engineering teardown" §三: QK
+//         normalisation, then interleaved rotary on the first dims): the two threads of a
+//         row add their halves' sums of squares, scale by rsqrt(mean + eps) and the gain,
+//         and rotate the pairs (2j, 2j+1) of dims [0, rot) by the position's angle.
 // Q K^T of tile j+1 overlaps the softmax of tile j.  The tensor pipe runs its MMAs in
 // issue order (Q K^T j+1, P V j, Q K^T j+2, ...), so P V j has read P_j before
 // Q K^T j+2 overwrites that buffer: no barrier is needed for the reuse.  TMEM: the two
@@ -75,7 +80,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __nv_bfloat16* __restrict__ q, int ld_q, const __grid_constant__ CUtensorMap tK,
                    const __grid_constant__ CUtensorMap tV, const __nv_bfloat16* __restrict__ gate, int ld_gate,
                    __nv_bfloat16* __restrict__ out, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
-                   float scale_log2, int QT) {
+                   float scale_log2, int QT, const __nv_bfloat16* __restrict__ q_norm, float eps, int rot,
+                   float rope_base, const float2* __restrict__ rope_tab, int tab_pos0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                                 // Q quarters: dims [64c, 64c + 64) at c * Q_BYTES / 4
@@ -244,11 +250,70 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     {
       const bool ok = q0 + qi < Tq;
       const uint4* src = reinterpret_cast<const uint4*>(q + ((long)b * Tq + (ok ? q0 + qi : 0)) * ld_q + (long)h * AT_D);
-#pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        const int dim = 128 * half + 8 * c;
-        const uint4 v4 = ok ? src[dim >> 3] : make_uint4(0, 0, 0, 0);
+      auto put = [&](int dim, uint4 v4) {
         *reinterpret_cast<uint4*>(sQ + (dim >> 6) * (Q_BYTES / 4) + r * 128 + ((((dim & 63) >> 3) ^ (r & 7)) << 4)) = v4;
+      };
+      if (!q_norm) {
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          const int dim = 128 * half + 8 * c;
+          put(dim, ok ? src[dim >> 3] : make_uint4(0, 0, 0, 0));
+        }
+      } else {
+        // raw row: this half's sum of squares, exchanged with the other half's thread
+        float ss = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          float x8[8];
+          load8(reinterpret_cast<const __nv_bfloat16*>(src) + 128 * half + 8 * c, x8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(x8[e], x8[e], ss);
+        }
+        xsum[half * AT_M + r] = ok ? ss : 0.f;
+        asm volatile("bar.sync 1, 256;" ::: "memory");     // the 256 softmax threads
+        const float inv = rsqrtf((xsum[r] + xsum[AT_M + r]) * (1.f / AT_D) + eps);
+        asm volatile("bar.sync 1, 256;" ::: "memory");     // both read before xsum is reused
+        const int pos = qpos;
+#pragma unroll 2
+        for (int c = 0; c < 16; ++c) {
+          const int dim = 128 * half + 8 * c;
+          float x8[8], g8[8];
+          load8(reinterpret_cast<const __nv_bfloat16*>(src) + dim, x8);
+          load8(q_norm + dim, g8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x8[e] = ok ? x8[e] * inv * g8[e] : 0.f;
+          if (dim < rot) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int jp = (dim + e) >> 1;
+              float cs, sn;
+              if (rope_tab) {
+                const float2 t2 = rope_tab[(long)(ok ? pos - tab_pos0 : 0) * (rot / 2) + jp];
+                cs = t2.x;
+                sn = t2.y;
+              } else {
+                const double theta = pow((double)rope_base, -2.0 * (double)jp / (double)rot);
+                double ang = (double)pos * theta;
+                ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
+                double sd, cd;
+                sincos(ang, &sd, &cd);
+                cs = (float)cd;
+                sn = (float)sd;
+              }
+              const float a0 = x8[e], a1 = x8[e + 1];
+              x8[e] = a0 * cs - a1 * sn;
+              x8[e + 1] = a0 * sn + a1 * cs;
+            }
+          }
+          uint4 v4;
+          uint32_t* pw = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(x8[2 * e], x8[2 * e + 1]);
+            pw[e] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          put(dim, v4);
+        }
       }
       fence_proxy_async();                            // generic stores -> tensor-core reads
       mbar_arrive(q_full);
@@ -387,7 +452,7 @@ bool gqa_tc_supported(int dh, int dtype, const void* q, int ld_q, const void* ga
 
 cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate,
                         int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
-                        cudaStream_t s) {
+                        cudaStream_t s, const QNorm* qn) {
   using namespace tc;
   const int rep = Hq / Hkv;
   if (rep < 1 || AT_M % rep != 0) return cudaErrorNotSupported;
@@ -401,8 +466,11 @@ cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, i
   }
   dim3 grid((Tq + QT - 1) / QT, Hkv, B);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)AT_D);
-  attn_tc_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>((const __nv_bfloat16*)q, ld_q, mK, mV, (const __nv_bfloat16*)gate, ld_gate,
-                                            (__nv_bfloat16*)out, Tq, Tkv, q_off, Hq, Hkv, causal, scale_log2, QT);
+  if (qn && qn->rot > AT_D / 2) return cudaErrorNotSupported;   // rotary dims must lie in the first half
+  attn_tc_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>(
+      (const __nv_bfloat16*)q, ld_q, mK, mV, (const __nv_bfloat16*)gate, ld_gate, (__nv_bfloat16*)out, Tq, Tkv, q_off,
+      Hq, Hkv, causal, scale_log2, QT, qn ? (const __nv_bfloat16*)qn->gain : nullptr, qn ? qn->eps : 0.f,
+      qn ? qn->rot : 0, qn ? qn->base : 1.f, qn ? qn->tab : nullptr, qn ? qn->tab_pos0 : 0);
   return cudaGetLastError();
 }
 

@@ -63,6 +63,14 @@ static loop_status check_config(const loop_config* c) {
   REQUIRE(c->sinkhorn_iters >= 0, LOOP_ERR_INVALID_ARG, "sinkhorn_iters must be >= 0");
   REQUIRE(gdn_supported(c->gdn_dk, c->gdn_dv) && c->gdn_heads > 0, LOOP_ERR_UNSUPPORTED,
           "GDN head sizes (dk, dv) must be (64, 64) or (128, 128)");
+  REQUIRE(c->gdn_variant == 0 || c->gdn_variant == 1, LOOP_ERR_INVALID_ARG, "gdn_variant must be 0 or 1");
+  if (c->gdn_variant == 0)
+    REQUIRE(c->gdn_v_heads == 0 || c->gdn_v_heads == c->gdn_heads, LOOP_ERR_INVALID_ARG,
+            "the plain GDN has as many value heads as key heads");
+  else
+    REQUIRE(gdn_variant_supported(c->gdn_heads, c->gdn_v_heads ? c->gdn_v_heads : c->gdn_heads, c->gdn_dk, c->gdn_dv,
+                                  c->gdn_conv),
+            LOOP_ERR_UNSUPPORTED, "GDN variant: value heads a multiple of the key heads, conv 4");
   REQUIRE(c->gdn_chunk == 64, LOOP_ERR_UNSUPPORTED, "GDN chunk must be 64");
   REQUIRE(gqa_supported(c->fa_head_dim, c->fa_q_heads, c->fa_kv_heads), LOOP_ERR_UNSUPPORTED,
           "FA head dim must be 64, 128 or 256 and Hq a multiple of Hkv (ratio <= 32)");
@@ -109,6 +117,7 @@ loop_status loop_model_create(const loop_config* cfg, const loop_weights* w, loo
     const bool fa = (l % cfg->group) == cfg->group - 1;
     bool ok = L.attn_norm && L.w_in && L.w_out && L.ffn_norm && L.w_gate && L.w_up && L.w_down;
     ok = ok && (fa ? (L.q_norm && L.k_norm) : (L.gdn_a_bias && L.gdn_b_bias));
+    if (!fa && cfg->gdn_variant == 1) ok = ok && L.gdn_conv_w && L.gdn_o_norm;
     if (l >= cfg->loop_start && l < cfg->loop_end && cfg->loop_passes > 0) ok = ok && L.mhc_w_r && L.mhc_b_r;
     if (!ok) return fail(LOOP_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": a required weight pointer is NULL");
   }
@@ -128,7 +137,10 @@ loop_status loop_model_create(const loop_config* cfg, const loop_weights* w, loo
     }
   }
   m->esize = cfg->dtype == LOOP_BF16 ? 2 : 4;
-  m->in_gdn = 2 * cfg->gdn_heads * cfg->gdn_dk + cfg->gdn_heads * cfg->gdn_dv + 2 * cfg->gdn_heads;
+  m->gdn_hv = cfg->gdn_v_heads ? cfg->gdn_v_heads : cfg->gdn_heads;
+  m->gdn_ch = 2 * cfg->gdn_heads * cfg->gdn_dk + m->gdn_hv * cfg->gdn_dv;
+  m->in_gdn = cfg->gdn_variant == 1 ? m->gdn_ch + m->gdn_hv * cfg->gdn_dv + 2 * m->gdn_hv
+                                    : 2 * cfg->gdn_heads * cfg->gdn_dk + cfg->gdn_heads * cfg->gdn_dv + 2 * cfg->gdn_heads;
   m->in_fa = 2 * cfg->fa_q_heads * cfg->fa_head_dim + 2 * cfg->fa_kv_heads * cfg->fa_head_dim;
   *out = m;
   return LOOP_OK;
@@ -150,10 +162,13 @@ loop_status loop_cache_create(const loop_model* m, int batch, int max_tokens, lo
   k->batch = batch;
   k->max_tokens = max_tokens;
   k->kv_slab_elems = (size_t)batch * c.fa_kv_heads * max_tokens * c.fa_head_dim;
-  k->state_elems = (size_t)batch * c.gdn_heads * c.gdn_dv * c.gdn_dk;
+  k->state_elems = (size_t)batch * m->gdn_hv * c.gdn_dv * c.gdn_dk;
+  k->conv_elems = c.gdn_variant == 1 ? (size_t)batch * (c.gdn_conv - 1) * m->gdn_ch : 0;
   cudaError_t e = k->kv.ensure(std::max<size_t>(256, (size_t)m->n_fa * 2 * k->kv_slab_elems * m->esize));
   if (e == cudaSuccess) e = k->state.ensure(std::max<size_t>(256, (size_t)m->n_gdn * k->state_elems * sizeof(float)));
+  if (e == cudaSuccess) e = k->conv.ensure(std::max<size_t>(256, (size_t)m->n_gdn * k->conv_elems * m->esize));
   if (e == cudaSuccess) e = cudaMemset(k->state.p, 0, k->state.bytes);
+  if (e == cudaSuccess) e = cudaMemset(k->conv.p, 0, k->conv.bytes);
   if (e != cudaSuccess) {
     delete k;
     return cuda_fail(e, "cache allocation");
@@ -165,6 +180,7 @@ loop_status loop_cache_create(const loop_model* m, int batch, int max_tokens, lo
 loop_status loop_cache_reset(loop_cache* c) {
   REQUIRE(c, LOOP_ERR_INVALID_ARG, "cache is NULL");
   cudaError_t e = cudaMemset(c->state.p, 0, c->state.bytes);
+  if (e == cudaSuccess) e = cudaMemset(c->conv.p, 0, c->conv.bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cache reset");
   c->len = 0;
   return LOOP_OK;
@@ -192,7 +208,7 @@ loop_status loop_cache_bytes(const loop_cache* c, size_t* kv_bytes, size_t* stat
   REQUIRE(c, LOOP_ERR_INVALID_ARG, "cache is NULL");
   const loop_model* m = c->model;
   if (kv_bytes) *kv_bytes = (size_t)m->n_fa * 2 * c->kv_slab_elems * m->esize;
-  if (state_bytes) *state_bytes = (size_t)m->n_gdn * c->state_elems * sizeof(float);
+  if (state_bytes) *state_bytes = (size_t)m->n_gdn * (c->state_elems * sizeof(float) + c->conv_elems * m->esize);
   return LOOP_OK;
 }
 
@@ -287,6 +303,33 @@ loop_status gdn_step(const void* q, const void* k, const void* v, const float* g
   return launched(lk::gdn_step(q, k, v, g, beta, state, out, B, H, dk, dv, scale, dtype, S(stream)), "gdn_step");
 }
 
+loop_status gdn_conv_prep(const void* P, int ld_p, const void* conv_w, void* conv_state, const float* a_bias,
+                          const float* b_bias, void* q, void* k, void* v, float* g, float* beta, int B, int T, int Hk,
+                          int Hv, int dk, int dv, int conv, float eps, int dtype, void* stream) {
+  REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
+  REQUIRE(B >= 0 && T >= 0, LOOP_ERR_INVALID_ARG, "negative size");
+  if (B == 0 || T == 0) return LOOP_OK;
+  REQUIRE(P && conv_w && conv_state && a_bias && b_bias && q && k && v && g && beta, LOOP_ERR_INVALID_ARG,
+          "NULL argument");
+  REQUIRE(gdn_variant_supported(Hk, Hv, dk, dv, conv), LOOP_ERR_UNSUPPORTED,
+          "Hv a multiple of Hk, (dk, dv) (64, 64) or (128, 128), conv 4");
+  REQUIRE(ld_p >= 2 * Hk * dk + 2 * Hv * dv + 2 * Hv, LOOP_ERR_SHAPE, "ld_p smaller than the projection width");
+  return launched(lk::gdn_conv_prep(P, ld_p, conv_w, conv_state, a_bias, b_bias, q, k, v, g, beta, B, T, Hk, Hv, dk,
+                                    dv, conv, eps, dtype, S(stream)),
+                  "gdn_conv_prep");
+}
+
+loop_status gdn_gated_norm(const void* o, const void* z, int ld_z, const void* w, void* y, int M, int H, int dv,
+                           float eps, int dtype, void* stream) {
+  REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
+  REQUIRE(M >= 0 && H > 0 && dv > 0, LOOP_ERR_INVALID_ARG, "bad size");
+  if (M == 0) return LOOP_OK;
+  REQUIRE(o && z && w && y, LOOP_ERR_INVALID_ARG, "NULL argument");
+  REQUIRE(dv % 32 == 0 && dv <= 256, LOOP_ERR_UNSUPPORTED, "dv must be a multiple of 32, <= 256");
+  REQUIRE(ld_z >= H * dv, LOOP_ERR_SHAPE, "ld_z smaller than H*dv");
+  return launched(lk::gdn_gated_norm(o, z, ld_z, w, y, M, H, dv, eps, dtype, S(stream)), "gdn_gated_norm");
+}
+
 loop_status gdn_prep(const void* P, int ld_p, const float* a_bias, const float* b_bias, void* q, void* k, void* v,
                      float* g, float* beta, int M, int H, int dk, int dv, float eps, int dtype, void* stream) {
   REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
@@ -315,13 +358,30 @@ loop_status gqa_attn(const void* q, int ld_q, const void* k, const void* v, int 
                   "gqa_attn");
 }
 
+loop_status gqa_attn_fused_q(const void* q, int ld_q, const void* q_norm, int rotary_dims, float rope_base, float eps,
+                             const void* k, const void* v, int kv_cap, const void* gate, int ld_gate, void* out, int B,
+                             int Tq, int Tkv, int q_off, int Hq, int Hkv, int dh, int causal, int dtype, void* stream) {
+  bool empty = false;
+  loop_status st = gqa_check_args("gqa_attn_fused_q", q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq,
+                                  Hkv, dh, causal, dtype, &empty);
+  if (st != LOOP_OK || empty) return st;
+  REQUIRE(q_norm, LOOP_ERR_INVALID_ARG, "q_norm is NULL");
+  REQUIRE(rotary_dims >= 0 && rotary_dims % 2 == 0 && rotary_dims <= dh / 2, LOOP_ERR_INVALID_ARG,
+          "rotary_dims must be even and <= dh / 2");
+  REQUIRE(eps >= 0.f && rope_base > 0.f, LOOP_ERR_INVALID_ARG, "eps >= 0 and rope_base > 0 required");
+  const QNorm qn{q_norm, rotary_dims, rope_base, eps, nullptr, 0};
+  return launched(lk::gqa_attn(q, ld_q, k, v, kv_cap, gate, ld_gate, out, B, Tq, Tkv, q_off, Hq, Hkv, dh, causal,
+                               nullptr, dtype, S(stream), &qn),
+                  "gqa_attn_fused_q");
+}
+
 loop_status fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out, void* k_cache,
                     void* v_cache, int kv_cap, int B, int T, int pos0, int Hq, int Hkv, int dh, int rotary_dims,
                     float rope_base, float eps, int dtype, void* stream) {
   REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
   REQUIRE(B >= 0 && T >= 0 && pos0 >= 0, LOOP_ERR_INVALID_ARG, "negative size");
   if (B == 0 || T == 0) return LOOP_OK;
-  REQUIRE(P && q_norm && k_norm && q_out && k_cache && v_cache, LOOP_ERR_INVALID_ARG, "NULL argument");
+  REQUIRE(P && q_norm && k_norm && k_cache && v_cache, LOOP_ERR_INVALID_ARG, "NULL argument");
   REQUIRE(gqa_supported(dh, Hq, Hkv), LOOP_ERR_UNSUPPORTED, "head dim or head ratio not supported");
   REQUIRE(pos0 + T <= kv_cap, LOOP_ERR_CAPACITY, "positions past the slab capacity");
   REQUIRE(ld_p >= 2 * Hq * dh + 2 * Hkv * dh, LOOP_ERR_SHAPE, "ld_p smaller than the projection width");

@@ -327,22 +327,24 @@ size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv) {
   return (size_t)B * H * chunks * (GDN_C * (dk + dv) + GDN_C * GDN_C + GDN_C) * sizeof(float);
 }
 
-// Workspace block of the tensor-core scan (bf16 models): W and P in bf16 (they are MMA
-// operands), U' and G in fp32.  Byte offsets within one (b, h, chunk) block.
+// Workspace block of the tensor-core scan (bf16 models), byte offsets within one
+// (b, h, chunk) block: the left factor Aw = (I + A)^-1 diag(beta gamma) as two bf16
+// terms, hi rows 0..63 then lo rows 64..127 of a [128][64] array (the scan forms
+// W S^T = Aw (K S^T), so W itself is never rounded); U' fp32 [64][dv]; P bf16 [64][64];
+// G fp32 [64].
 template <int DK, int DV>
 struct GdnWsB {
-  static constexpr int W_OFF = 0, U_OFF = GDN_C * DK * 2, P_OFF = U_OFF + GDN_C * DV * 4,
+  static constexpr int AW_OFF = 0, U_OFF = 2 * GDN_C * GDN_C * 2, P_OFF = U_OFF + GDN_C * DV * 4,
                        G_OFF = P_OFF + GDN_C * GDN_C * 2, BYTES = G_OFF + GDN_C * 4;
 };
 
-template <typename T, int DK, int DV, bool WB>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ g,
                                                         const float* __restrict__ beta, float* __restrict__ ws,
                                                         int T_len, int H, int n_chunks) {
   constexpr int C = GDN_C, CP = GDN_C + 4;
   using WL = GdnWs<DK, DV>;
-  using WLB = GdnWsB<DK, DV>;
   extern __shared__ float sm[];
   float* Kt = sm;                 // [DK][CP] keys, transposed
   float* Qt = Kt + DK * CP;       // [DK][CP] queries, transposed
@@ -352,7 +354,6 @@ __global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int c0 = c * C, n = min(C, T_len - c0);
   float* blk = ws + (((long)b * H + h) * n_chunks + c) * WL::FLOATS;
-  uint8_t* blkb = (uint8_t*)ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
   for (int idx = tid; idx < C * DK; idx += 256) {
     const int r = idx / DK, j = idx % DK;
     float kv = 0.f, qv = 0.f;
@@ -382,10 +383,7 @@ __global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__
     Gs[2 * tid + 1] = x;
   }
   __syncthreads();
-  if (tid < C) {
-    if (WB) reinterpret_cast<float*>(blkb + WLB::G_OFF)[tid] = Gs[tid];
-    else blk[WL::G_OFF + tid] = Gs[tid];
-  }
+  if (tid < C) blk[WL::G_OFF + tid] = Gs[tid];
   {
     // 4 x 4 blocks of K K^T and Q K^T on and below the diagonal
     const int r0 = (tid >> 4) * 4, s0 = (tid & 15) * 4;
@@ -423,13 +421,7 @@ __global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__
         pv[e] = aq[a][e] * dec;
       }
       *reinterpret_cast<float4*>(As + r * CP + s0) = make_float4(av[0], av[1], av[2], av[3]);
-      if (WB) {
-        __nv_bfloat162* pb = reinterpret_cast<__nv_bfloat162*>(blkb + WLB::P_OFF + (r * C + s0) * 2);
-        pb[0] = __floats2bfloat162_rn(pv[0], pv[1]);
-        pb[1] = __floats2bfloat162_rn(pv[2], pv[3]);
-      } else {
-        *reinterpret_cast<float4*>(blk + WL::P_OFF + r * C + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
-      }
+      *reinterpret_cast<float4*>(blk + WL::P_OFF + r * C + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
     }
   }
   __syncthreads();
@@ -458,15 +450,7 @@ __global__ void __launch_bounds__(256, 2) gdn_intra_kernel(const T* __restrict__
       }
       x[r] = acc;
     }
-    if (WB && j < DK) {
-      __nv_bfloat16* wd = reinterpret_cast<__nv_bfloat16*>(blkb + WLB::W_OFF) + j;
-#pragma unroll
-      for (int r = 0; r < C; ++r) wd[r * DK] = __float2bfloat16(x[r]);
-    } else if (WB) {
-      float* ud = reinterpret_cast<float*>(blkb + WLB::U_OFF) + (j - DK);
-#pragma unroll
-      for (int r = 0; r < C; ++r) ud[r * DV] = x[r];
-    } else {
+    {
       float* dst = j < DK ? blk + WL::W_OFF + j : blk + WL::U_OFF + (j - DK);
       const int stride = j < DK ? DK : DV;
 #pragma unroll
@@ -651,44 +635,57 @@ __global__ void __launch_bounds__(256) gdn_scan_kernel(const T* __restrict__ q, 
 
 
 // ------------------------------------------------------------------ tensor-core sequential pass (bf16)
-// The same recurrence as gdn_scan_kernel with the three per-chunk products on the tensor
-// cores (mma.sync m16n8k16, bf16 operands, fp32 accumulation):
-//   U  = U' - W S^T          (64 x 16, K = dk)      A = W,  B = S (bf16 copy)
-//   O  = gamma Q S^T + P U   (64 x 16, K = dk, 64)  A = Q, P; B = S, U
-//   S <- exp(G_last) S + (exp(G_last - G) U)^T K   (16 x dk, K = 64)
+// The same recurrence as gdn_scan_kernel with the per-chunk products on the tensor cores
+// (mma.sync m16n8k16, bf16 operands, fp32 accumulation):
+//   Y  = K S^T               (64 x 16, K = dk)      A = K (exact),  B = S as bf16 hi + lo
+//   U  = U' - Aw Y           (64 x 16, K = 64)      A = Aw hi + lo, B = Y hi + lo   (W S^T = Aw K S^T)
+//   O  = gamma Q S^T + P U   (64 x 16, K = dk, 64)  A = Q, P; B = S hi, U (output: bf16 operands)
+//   S <- exp(G_last) S + (exp(G_last - G) U)^T K   (16 x dk, K = 64)  A = as bf16 hi + lo, B = K
+// Every product on the state's path has exact operands or operands carried as two bf16
+// terms (hi + lo, relative error ~2^-17; the lo x lo term is dropped), so the state is
+// updated with fp32-grade accuracy; only the output products use single bf16 operands.
 // The fp32 state lives in registers as the accumulator of the last product; each warp
 // owns dk/64 8-column tiles of the 16 state rows of this CTA.
 __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float x, float y) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
 }
+// x ~ hi + lo as two bf16 pairs
+__device__ __forceinline__ void st_bf2_split(__nv_bfloat16* hi, __nv_bfloat16* lo, float x, float y) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 f = __bfloat1622float2(h);
+  *reinterpret_cast<__nv_bfloat162*>(hi) = h;
+  *reinterpret_cast<__nv_bfloat162*>(lo) = __floats2bfloat162_rn(x - f.x, y - f.y);
+}
 
-// Shared-memory plan of the tensor-core scan.  A chunk's W, Q, K (64 x dk bf16) and P
-// (64 x 64 bf16) arrive by TMA as 64-column halves of [64 rows x 128 B] with the 128-byte
-// swizzle (16-byte chunk j of row r stored at j ^ (r & 7)); U' (this CTA's 16 columns,
-// fp32) and G (fp32) as plain boxes.  Nine tile loads per chunk, completing on the
-// stage's mbarrier.
+// Shared-memory plan of the tensor-core scan.  A chunk's Aw (hi and lo, [128 rows x 64]),
+// Q, K (64 x dk) and P (64 x 64) arrive by TMA as 64-column pieces of [rows x 128 B] with
+// the 128-byte swizzle (16-byte chunk j of row r stored at j ^ (r & 7)); U' (this CTA's 16
+// columns, fp32) and G (fp32) as plain boxes.  Seven or nine tile loads per chunk,
+// completing on the stage's mbarrier.
 template <int DK, int DV>
 struct ScanTc {
   static constexpr int C = GDN_C, DVS = 16, KP = DK + 8, UP = DVS + 8;
-  static constexpr int HALF = C * 128;                       // one 64-column half, 8 KB
-  static constexpr int W_B = (DK / 64) * HALF, Q_B = W_B, K_B = W_B, P_B = HALF, UPF_B = C * DVS * 4, G_B = C * 4;
-  static constexpr int TX = W_B + Q_B + K_B + P_B + UPF_B + G_B;     // bytes per chunk
+  static constexpr int HALF = C * 128;                       // one 64-column piece of 64 rows, 8 KB
+  static constexpr int AW_B = 2 * HALF, Q_B = (DK / 64) * HALF, K_B = Q_B, P_B = HALF, UPF_B = C * DVS * 4,
+                       G_B = C * 4;
+  static constexpr int TX = AW_B + Q_B + K_B + P_B + UPF_B + G_B;    // bytes per chunk
   static constexpr int STAGE = (TX + 1023) / 1024 * 1024;            // swizzled tiles: 1024-byte aligned
   static constexpr int SB_B = DVS * KP * 2, UB_B = C * UP * 2;
   static constexpr int NSTAGE = 3;                           // chunks in flight: two ahead of the one in use
-  static constexpr int BAR_OFF = NSTAGE * STAGE + SB_B + 2 * UB_B;   // NSTAGE mbarriers, then an abort flag
+  // state hi, lo; U; exp(G_last - G) U hi, lo; Y hi, lo
+  static constexpr int BAR_OFF = NSTAGE * STAGE + 2 * SB_B + 5 * UB_B;   // NSTAGE mbarriers, then an abort flag
   static constexpr size_t BYTES = (size_t)BAR_OFF + 8 * NSTAGE + 16 + 1024;   // + alignment slack
   static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
 };
 
 // Byte offset of bf16 element (row, col) (col a multiple of 8) in a tile stored as 64-column
-// halves of [GDN_C rows x 128 B] with the 128-byte swizzle.
+// pieces of [GDN_C rows x 128 B] with the 128-byte swizzle (rows < 64 per piece).
 __device__ __forceinline__ uint32_t sw_off(int row, int col) {
   return (uint32_t)((col >> 6) * (GDN_C * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap mW,
+__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap mA,
                                                           const __grid_constant__ CUtensorMap mP,
                                                           const __grid_constant__ CUtensorMap mU,
                                                           const __grid_constant__ CUtensorMap mG,
@@ -701,9 +698,13 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
   constexpr int NT3 = DK / 64;                               // state column tiles per warp
   extern __shared__ __align__(16) uint8_t smb_raw[];
   uint8_t* smb = (uint8_t*)(((uintptr_t)smb_raw + 1023) & ~(uintptr_t)1023);
-  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + L::NSTAGE * L::STAGE);  // [DVS][KP] bf16 copy of the state slice
-  __nv_bfloat16* Ub = Sb + DVS * KP;                         // [C][UP] U
-  __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U
+  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + L::NSTAGE * L::STAGE);  // [DVS][KP] state slice, bf16 hi part
+  __nv_bfloat16* Sl = Sb + DVS * KP;                         // ... and lo part
+  __nv_bfloat16* Ub = Sl + DVS * KP;                         // [C][UP] U (bf16, output product)
+  __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U, hi
+  __nv_bfloat16* Uel = Ueb + C * UP;                         // ... lo
+  __nv_bfloat16* Yh = Uel + C * UP;                          // [C][UP] Y = K S^T, hi
+  __nv_bfloat16* Yl = Yh + C * UP;                           // ... lo
   uint64_t* full = reinterpret_cast<uint64_t*>(smb + L::BAR_OFF);   // a chunk's tiles landed, per stage
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + L::NSTAGE);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
@@ -711,7 +712,7 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
     for (int i = 0; i < L::NSTAGE; ++i) tc::mbar_init(tc::smem_u32(full + i), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mW) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mA) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mQ) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mK) : "memory");
   }
@@ -726,24 +727,24 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
     st[j][1] = Sg[gq * DK + col + 1];
     st[j][2] = Sg[(gq + 8) * DK + col];
     st[j][3] = Sg[(gq + 8) * DK + col + 1];
-    st_bf2(Sb + gq * KP + col, st[j][0], st[j][1]);
-    st_bf2(Sb + (gq + 8) * KP + col, st[j][2], st[j][3]);
+    st_bf2_split(Sb + gq * KP + col, Sl + gq * KP + col, st[j][0], st[j][1]);
+    st_bf2_split(Sb + (gq + 8) * KP + col, Sl + (gq + 8) * KP + col, st[j][2], st[j][3]);
   }
 
-  // one thread: the chunk's nine tiles (rows past the sequence end read as zeros)
+  // one thread: the chunk's tiles (rows past the sequence end read as zeros)
   auto issue = [&](int c, int bi) {
     uint8_t* base = smb + bi * L::STAGE;
     const int blk = ((b * H + h) * n_chunks + c);
     const uint32_t fb = tc::smem_u32(full + bi);
     tc::fence_proxy_async();                                 // earlier generic reads of this stage first
     tc::mbar_expect_tx(fb, (uint32_t)L::TX);
+    tc::tma_load_3d(tc::smem_u32(base), &mA, fb, 0, 0, blk);
 #pragma unroll
     for (int hf = 0; hf < DK / 64; ++hf) {
-      tc::tma_load_3d(tc::smem_u32(base + hf * L::HALF), &mW, fb, hf * 64, 0, blk);
-      tc::tma_load_4d(tc::smem_u32(base + L::W_B + hf * L::HALF), &mQ, fb, hf * 64, h, c * C, b);
-      tc::tma_load_4d(tc::smem_u32(base + L::W_B + L::Q_B + hf * L::HALF), &mK, fb, hf * 64, h, c * C, b);
+      tc::tma_load_4d(tc::smem_u32(base + L::AW_B + hf * L::HALF), &mQ, fb, hf * 64, h, c * C, b);
+      tc::tma_load_4d(tc::smem_u32(base + L::AW_B + L::Q_B + hf * L::HALF), &mK, fb, hf * 64, h, c * C, b);
     }
-    const int off_p = L::W_B + L::Q_B + L::K_B;
+    const int off_p = L::AW_B + L::Q_B + L::K_B;
     tc::tma_load_3d(tc::smem_u32(base + off_p), &mP, fb, 0, 0, blk);
     tc::tma_load_3d(tc::smem_u32(base + off_p + L::P_B), &mU, fb, i0, 0, blk);
     tc::tma_load_2d(tc::smem_u32(base + off_p + L::P_B + L::UPF_B), &mG, fb, 0, blk);
@@ -763,42 +764,63 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
     __syncthreads();
     if (tid == 0 && c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
     const uint8_t* base = smb + bi * L::STAGE;
-    const uint8_t* Wb = base;                                // swizzled tiles (sw_off)
-    const uint8_t* Qb = base + L::W_B;
-    const uint8_t* Kb = base + L::W_B + L::Q_B;
-    const uint8_t* Pb = base + L::W_B + L::Q_B + L::K_B;
-    const float* Upf = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B);
-    const float* Gs = (const float*)(base + L::W_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
+    const uint8_t* Awb = base;                               // swizzled tiles (sw_off)
+    const uint8_t* Qb = base + L::AW_B;
+    const uint8_t* Kb = base + L::AW_B + L::Q_B;
+    const uint8_t* Pb = base + L::AW_B + L::Q_B + L::K_B;
+    const float* Upf = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B);
+    const float* Gs = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
     const int c0 = c * C, n = min(C, T_len - c0);
     const float Glast = Gs[C - 1];
     // decay factors depend on G only: computed while the MMA chain below runs
     const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
     const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]), gl = expf(Glast);
-    // phase 1 + 2a: W S^T and Q S^T share the B operand; even and odd k-steps go to
-    // separate accumulators, halving the dependent MMA chain on the sequential path
-    float cu[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
-    float cu1[4] = {0.f, 0.f, 0.f, 0.f}, cq1[4] = {0.f, 0.f, 0.f, 0.f};
+    // phase 1a: Y = K S^T (S as hi + lo) and Q S^T (hi) share the B operand; the lo term and
+    // the odd k-steps go to separate accumulators (short dependent MMA chains)
+    float cy[4] = {0.f, 0.f, 0.f, 0.f}, cy1[4] = {0.f, 0.f, 0.f, 0.f}, cyl[4] = {0.f, 0.f, 0.f, 0.f};
+    float cq[4] = {0.f, 0.f, 0.f, 0.f}, cq1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < DK / 16; ++ks) {
-      uint32_t aw[4], aq[4], bs[2];
-      ldsm_x4(aw, Wb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
+      uint32_t ak[4], aq[4], bs[2], bl[2];
+      ldsm_x4(ak, Kb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
       ldsm_x4(aq, Qb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x2(bs, Sb + (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8);
-      mma16816((ks & 1) ? cu1 : cu, aw, bs);
+      const int srow = (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8;
+      ldsm_x2(bs, Sb + srow);
+      ldsm_x2(bl, Sl + srow);
+      mma16816((ks & 1) ? cy1 : cy, ak, bs);
+      mma16816(cyl, ak, bl);
       mma16816((ks & 1) ? cq1 : cq, aq, bs);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      cu[e] += cu1[e];
+      cy[e] += cy1[e] + cyl[e];
       cq[e] += cq1[e];
     }
+    st_bf2_split(Yh + r0 * UP + ic, Yl + r0 * UP + ic, cy[0], cy[1]);
+    st_bf2_split(Yh + r1 * UP + ic, Yl + r1 * UP + ic, cy[2], cy[3]);
+    __syncthreads();
+    // phase 1b: W S^T = Aw Y with Aw and Y both as hi + lo (lo x lo dropped)
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cw1[4] = {0.f, 0.f, 0.f, 0.f}, cwl[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      uint32_t ah[4], al[4], yh[2], yl[2];
+      ldsm_x4(ah, Awb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
+      ldsm_x4(al, Awb + L::HALF + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
+      ldsm_x2_t(yh, Yh + (ks * 16 + (lane & 15)) * UP + nt * 8);
+      ldsm_x2_t(yl, Yl + (ks * 16 + (lane & 15)) * UP + nt * 8);
+      mma16816((ks & 1) ? cw1 : cw, ah, yh);
+      mma16816(cwl, ah, yl);
+      mma16816(cwl, al, yh);
+    }
     {
-      const float u00 = Upf[r0 * DVS + ic] - cu[0], u01 = Upf[r0 * DVS + ic + 1] - cu[1];
-      const float u10 = Upf[r1 * DVS + ic] - cu[2], u11 = Upf[r1 * DVS + ic + 1] - cu[3];
+      const float w00 = cw[0] + cw1[0] + cwl[0], w01 = cw[1] + cw1[1] + cwl[1];
+      const float w10 = cw[2] + cw1[2] + cwl[2], w11 = cw[3] + cw1[3] + cwl[3];
+      const float u00 = Upf[r0 * DVS + ic] - w00, u01 = Upf[r0 * DVS + ic + 1] - w01;
+      const float u10 = Upf[r1 * DVS + ic] - w10, u11 = Upf[r1 * DVS + ic + 1] - w11;
       st_bf2(Ub + r0 * UP + ic, u00, u01);
       st_bf2(Ub + r1 * UP + ic, u10, u11);
-      st_bf2(Ueb + r0 * UP + ic, u00 * e0, u01 * e0);
-      st_bf2(Ueb + r1 * UP + ic, u10 * e1, u11 * e1);
+      st_bf2_split(Ueb + r0 * UP + ic, Uel + r0 * UP + ic, u00 * e0, u01 * e0);
+      st_bf2_split(Ueb + r1 * UP + ic, Uel + r1 * UP + ic, u10 * e1, u11 * e1);
     }
     __syncthreads();
     // phase 2b: P U, then the outputs
@@ -823,32 +845,36 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
     for (int j = 0; j < NT3; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st[j][e] *= gl;
-    // the second half of the k-steps accumulates separately and is added at the end
-    float st1[NT3][4];
+    // the odd k-steps and the lo terms accumulate separately (independent MMA chains of
+    // depth 2) and are added at the end
+    float st1[NT3][4], sl0[NT3][4], sl1[NT3][4];
 #pragma unroll
     for (int j = 0; j < NT3; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st1[j][e] = 0.f;
+      for (int e = 0; e < 4; ++e) st1[j][e] = sl0[j][e] = sl1[j][e] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
-      uint32_t au[4];
-      ldsm_x4_t(au, Ueb + (ks * 16 + (lane >> 4) * 8 + (lane & 7)) * UP + ((lane >> 3) & 1) * 8);
+      uint32_t au[4], al[4];
+      const int urow = (ks * 16 + (lane >> 4) * 8 + (lane & 7)) * UP + ((lane >> 3) & 1) * 8;
+      ldsm_x4_t(au, Ueb + urow);
+      ldsm_x4_t(al, Uel + urow);
 #pragma unroll
       for (int j = 0; j < NT3; ++j) {
         uint32_t bk[2];
         ldsm_x2_t(bk, Kb + sw_off(ks * 16 + (lane & 15), (w * NT3 + j) * 8));
         mma16816((ks & 1) ? st1[j] : st[j], au, bk);
+        mma16816((ks & 1) ? sl1[j] : sl0[j], al, bk);
       }
     }
 #pragma unroll
     for (int j = 0; j < NT3; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st[j][e] += st1[j][e];
+      for (int e = 0; e < 4; ++e) st[j][e] += st1[j][e] + (sl0[j][e] + sl1[j][e]);
 #pragma unroll
     for (int j = 0; j < NT3; ++j) {
       const int col = (w * NT3 + j) * 8 + 2 * tq;
-      st_bf2(Sb + gq * KP + col, st[j][0], st[j][1]);
-      st_bf2(Sb + (gq + 8) * KP + col, st[j][2], st[j][3]);
+      st_bf2_split(Sb + gq * KP + col, Sl + gq * KP + col, st[j][0], st[j][1]);
+      st_bf2_split(Sb + (gq + 8) * KP + col, Sl + (gq + 8) * KP + col, st[j][2], st[j][3]);
     }
   }
 #pragma unroll
@@ -868,10 +894,11 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
 //   A[r][s] = beta_r exp(G_r - G_s) KK[r][s]  (s < r),  P[r][s] = exp(G_r - G_s) QK[r][s]  (s <= r)
 //   T = (I + A)^-1 in fp32: the four 16 x 16 diagonal blocks by substitution, then block
 //       row i = 1..3:  T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj
-//   W = (T diag(beta gamma)) K,  U' = (T diag(beta)) V   (gamma_s = exp(G_s); tensor cores,
-//       the fp32 left factor split into two bf16 terms, hi + lo, so its rounding error is
-//       about 2^-17 instead of 2^-9)
-// W, P (bf16), U', G (fp32) go to the workspace block the tensor-core sequential pass reads.
+//   Aw = T diag(beta gamma) (gamma_s = exp(G_s)) as two bf16 terms, hi + lo, so its
+//       rounding error is about 2^-17 instead of 2^-9; the sequential pass forms
+//       W S^T = Aw (K S^T) from it
+//   U' = (T diag(beta)) V   (tensor cores, the fp32 left factor split the same way)
+// Aw, P (bf16), U', G (fp32) go to the workspace block the tensor-core sequential pass reads.
 template <int DK, int DV>
 struct IntraTc {
   static constexpr int C = GDN_C;
@@ -915,7 +942,7 @@ __global__ void __launch_bounds__(256, 2)
   const int c0 = c * C, n = min(C, T_len - c0);
   uint8_t* blk = ws + (((long)b * H + h) * n_chunks + c) * (long)WLB::BYTES;
   __nv_bfloat16* Pg = reinterpret_cast<__nv_bfloat16*>(blk + WLB::P_OFF);
-  __nv_bfloat16* Wg = reinterpret_cast<__nv_bfloat16*>(blk + WLB::W_OFF);
+  __nv_bfloat16* Awg = reinterpret_cast<__nv_bfloat16*>(blk + WLB::AW_OFF);
   float* Ug = reinterpret_cast<float*>(blk + WLB::U_OFF);
 
   // ---- 1. the chunk's K, Q, V rows (zeros past the sequence end), decays and betas
@@ -1060,7 +1087,13 @@ __global__ void __launch_bounds__(256, 2)
   }
   __syncthreads();
 
-  // ---- 5. W = Aw K (bf16 out), U' = Au V (fp32 out): warp = (16-row tile, half of the columns)
+  // ---- 5. Aw (hi rows, then lo rows) to the workspace; U' = Au V (fp32 out): warp = (16-row
+  //         tile, half of the columns)
+  for (int e = tid; e < 2 * C * C / 8; e += 256) {           // 16-byte pieces of [2C][C]
+    const int r = e / (C / 8), p8 = e % (C / 8);
+    const __nv_bfloat16* src = (r < C ? Awh + r * SP : Awl + (r - C) * SP) + 8 * p8;
+    *reinterpret_cast<uint4*>(Awg + r * C + 8 * p8) = *reinterpret_cast<const uint4*>(src);
+  }
   {
     const int mt = w & 3, nh = w >> 2;
     auto product = [&](const __nv_bfloat16* Ah, const __nv_bfloat16* Al, const __nv_bfloat16* Bm, int BP, int NC,
@@ -1094,7 +1127,6 @@ __global__ void __launch_bounds__(256, 2)
         store(r0 + 8, col, acc[t2][2], acc[t2][3]);
       }
     };
-    product(Awh, Awl, Ks, KS, DK, [&](int r, int col, float x0, float x1) { st_bf2(Wg + r * DK + col, x0, x1); });
     product(Auh, Aul, Vs, VS, DV, [&](int r, int col, float x0, float x1) {
       *reinterpret_cast<float2*>(Ug + r * DV + col) = make_float2(x0, x1);
     });
@@ -1109,7 +1141,7 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
   const int n_chunks = (T_len + GDN_C - 1) / GDN_C;
   const size_t smem1 = (size_t)(2 * DK * (GDN_C + 4) + GDN_C * (GDN_C + 4) + 2 * GDN_C) * sizeof(float);
   constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;   // bf16: tensor-core sequential pass
-  auto k1 = gdn_intra_kernel<T, DK, DV, TC>;
+  auto k1 = gdn_intra_kernel<T, DK, DV>;
   auto k2 = gdn_scan_kernel<T, DK, DV, DVS>;
   auto k2t = gdn_scan_tc_kernel<DK, DV>;
   using L = ScanSmem<T, DK, DV, DVS>;
@@ -1141,22 +1173,23 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
     using WLB = GdnWsB<DK, DV>;
     const uint8_t* wsb = (const uint8_t*)workspace;
     const cuuint64_t nblk = (cuuint64_t)B * H * n_chunks, bs = (cuuint64_t)WLB::BYTES;
-    CUtensorMap mW, mP, mU, mG, mQ, mK;
-    const cuuint64_t dW[3] = {DK, GDN_C, nblk}, sW[2] = {DK * 2, bs};
+    CUtensorMap mA, mP, mU, mG, mQ, mK;
+    const cuuint64_t dA[3] = {GDN_C, 2 * GDN_C, nblk}, sA[2] = {GDN_C * 2, bs};
     const cuuint64_t dP[3] = {GDN_C, GDN_C, nblk}, sP[2] = {GDN_C * 2, bs};
     const cuuint64_t dU[3] = {DV, GDN_C, nblk}, sU[2] = {DV * 4, bs};
     const cuuint64_t dG[2] = {GDN_C, nblk}, sG[1] = {bs};
     const cuuint64_t dQ[4] = {DK, (cuuint64_t)H, (cuuint64_t)T_len, (cuuint64_t)B};
     const cuuint64_t sQ[3] = {DK * 2, (cuuint64_t)H * DK * 2, (cuuint64_t)T_len * H * DK * 2};
-    const cuuint32_t b64[3] = {64, GDN_C, 1}, bU[3] = {LT::DVS, GDN_C, 1}, bG[2] = {GDN_C, 1}, bQ[4] = {64, 1, GDN_C, 1};
+    const cuuint32_t b64[3] = {64, GDN_C, 1}, bA[3] = {64, 2 * GDN_C, 1}, bU[3] = {LT::DVS, GDN_C, 1},
+                     bG[2] = {GDN_C, 1}, bQ[4] = {64, 1, GDN_C, 1};
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    if (!tc::make_map_nd(&mW, BF, 3, wsb + WLB::W_OFF, dW, sW, b64, true) ||
+    if (!tc::make_map_nd(&mA, BF, 3, wsb + WLB::AW_OFF, dA, sA, bA, true) ||
         !tc::make_map_nd(&mP, BF, 3, wsb + WLB::P_OFF, dP, sP, b64, true) ||
         !tc::make_map_nd(&mU, F32, 3, wsb + WLB::U_OFF, dU, sU, bU, false) ||
         !tc::make_map_nd(&mG, F32, 2, wsb + WLB::G_OFF, dG, sG, bG, false) ||
         !tc::make_map_nd(&mQ, BF, 4, q, dQ, sQ, bQ, true) || !tc::make_map_nd(&mK, BF, 4, k, dQ, sQ, bQ, true))
       return cudaErrorNotSupported;
-    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>(mW, mP, mU, mG, mQ, mK, state, (__nv_bfloat16*)out, T_len, H,
+    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>(mA, mP, mU, mG, mQ, mK, state, (__nv_bfloat16*)out, T_len, H,
                                                           n_chunks, scale);
   } else
     k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,

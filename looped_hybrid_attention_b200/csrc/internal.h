@@ -52,6 +52,17 @@ cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g
                      float* state, void* out, int B, int H, int dk, int dv, float scale, int dtype,
                      cudaStream_t s);
 bool gdn_supported(int dk, int dv);
+// GDN variant (short causal conv + gated output norm; Hv value heads reading Hk key heads)
+bool gdn_variant_supported(int Hk, int Hv, int dk, int dv, int conv);
+// conv + SiLU on the q|k|v channels of P (rows q | k | v | z | a | b), L2 norm of q and k
+// (written once per value head that reads them), gates; then conv_state [B][conv-1][C]
+// becomes the last conv-1 inputs.  q, k [B*T, Hv, dk], v [B*T, Hv, dv], g, beta [B*T, Hv].
+cudaError_t gdn_conv_prep(const void* P, int ld_p, const void* conv_w, void* conv_state, const float* a_bias,
+                          const float* b_bias, void* q, void* k, void* v, float* g, float* beta, int B, int T, int Hk,
+                          int Hv, int dk, int dv, int conv, float eps, int dtype, cudaStream_t s);
+// y [M, H, dv] = RMSNorm(o) * w * silu(z) per head (y may equal o); z rows of stride ld_z.
+cudaError_t gdn_gated_norm(const void* o, const void* z, int ld_z, const void* w, void* y, long M, int H, int dv,
+                           float eps, int dtype, cudaStream_t s);
 
 // rope_tab: optional [T, rotary_dims/2] (cos, sin) table from rope_table (else fp64 in-kernel).
 cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_norm, void* q_out,
@@ -59,22 +70,36 @@ cudaError_t fa_prep(const void* P, int ld_p, const void* q_norm, const void* k_n
                     int Hkv, int dh, int rotary_dims, float rope_base, float eps, int dtype,
                     cudaStream_t s, const float2* rope_tab = nullptr);
 cudaError_t rope_table(float2* tab, int T, int pos0, int rot, float base, cudaStream_t s);
+struct QNorm;
+// qn: queries arrive raw (the input projection) and are QK-normed and rotated by the
+// tensor-core kernel as it stages them (bf16, head dim 256, Tq >= 16 only).
 cudaError_t gqa_attn(const void* q, int ld_q, const void* k, const void* v, int kv_cap,
                      const void* gate, int ld_gate, void* out, int B, int Tq, int Tkv, int q_off,
                      int Hq, int Hkv, int dh, int causal, void* workspace, int dtype,
-                     cudaStream_t s);
+                     cudaStream_t s, const QNorm* qn = nullptr);
 // Workspace bound for any Hkv and dtype (what loop_gqa_workspace_bytes promises).
 size_t gqa_workspace_bytes(int B, int Tq, int Tkv, int Hq, int dh);
 // Exact scratch bytes gqa_attn uses with a workspace for this call's shape (0: none).
 size_t gqa_scratch_bytes(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype);
 bool gqa_supported(int dh, int Hq, int Hkv);
 int gqa_launches(int B, int Tq, int Tkv, int Hq, int Hkv, int dh, int dtype, bool has_workspace);
+// Query normalisation and rotary applied by the attention kernel as it stages Q (q then is
+// the raw projection): gain [dh] (dtype), rotary dims (<= dh/2), base, eps, and an optional
+// cos/sin table whose row p - tab_pos0 holds position p (else fp64 in-kernel).  Query t
+// sits at position q_off + t.
+struct QNorm {
+  const void* gain;
+  int rot;
+  float base, eps;
+  const float2* tab;
+  int tab_pos0;
+};
 // tcgen05 flash attention (bf16, head dim 256); used for multi-token queries.
 bool gqa_tc_supported(int dh, int dtype, const void* q, int ld_q, const void* gate, int ld_gate, const void* k,
                       const void* v, int kv_cap);
 cudaError_t gqa_attn_tc(const void* q, int ld_q, const void* k, const void* v, int kv_cap, const void* gate,
                         int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv, int causal,
-                        cudaStream_t s);
+                        cudaStream_t s, const QNorm* qn = nullptr);
 
 // w_rt: optional [8, 2d] transposed copy of w_r (coalesced routing-map reads).
 cudaError_t mhc(int mode, const void* X_in, const void* F, const float* coeffs_in, const float* w_r,

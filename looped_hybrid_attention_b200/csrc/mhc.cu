@@ -40,16 +40,18 @@ namespace lk {
 // (one reciprocal each), and the last round writes the column-normalised matrix from
 // them.  The odds stay within exp(+-spread) and their product within exp(+-2 spread):
 // for spread <= 40 nothing overflows and the reciprocals come from the hardware
-// (rcp.approx, within about one ulp).  Wider spreads run the rounds literally with IEEE
-// divisions.
+// (rcp.approx, within about one ulp).  Wider spreads run the same rounds in the log domain
+// (each row, then each column, minus its log-sum-exp): in the linear domain the smallest
+// entries exp(-spread) would lose their precision to fp32 denormals (spread > ~87) or to
+// the row and column sums they are divided by.
 __device__ __forceinline__ float rcp_hw(float x) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
-__device__ __forceinline__ void sinkhorn2(float m[4], int iters, float spread) {
+__device__ __forceinline__ void sinkhorn2(float m[4], int iters) {
   if (iters <= 0) return;
-  if (spread <= 40.f) {
+  {
     float x = m[0] / m[1], y = m[2] / m[3];
 #pragma unroll 4
     for (int it = 1; it < iters; ++it) {
@@ -65,23 +67,36 @@ __device__ __forceinline__ void sinkhorn2(float m[4], int iters, float spread) {
     m[2] = b * r0;
     m[1] = px * r1;
     m[3] = py * r1;
-  } else {
-    for (int it = 0; it < iters; ++it) {
-      const float r0 = m[0] + m[1], r1 = m[2] + m[3];
-      m[0] /= r0; m[1] /= r0; m[2] /= r1; m[3] /= r1;
-      const float c0 = m[0] + m[2], c1 = m[1] + m[3];
-      m[0] /= c0; m[2] /= c0; m[1] /= c1; m[3] /= c1;
-    }
   }
+}
+
+// log(e^a + e^b)
+__device__ __forceinline__ float lse2(float a, float b) { return fmaxf(a, b) + log1pf(expf(-fabsf(a - b))); }
+
+// The rounds of sinkhorn2 in the log domain, from x = l - max l; writes exp(x).
+__device__ __forceinline__ void sinkhorn2_log(const float x_in[4], int iters, float m[4]) {
+  float x0 = x_in[0], x1 = x_in[1], x2 = x_in[2], x3 = x_in[3];
+  for (int it = 0; it < iters; ++it) {
+    const float r0 = lse2(x0, x1), r1 = lse2(x2, x3);
+    x0 -= r0; x1 -= r0; x2 -= r1; x3 -= r1;
+    const float c0 = lse2(x0, x2), c1 = lse2(x1, x3);
+    x0 -= c0; x2 -= c0; x1 -= c1; x3 -= c1;
+  }
+  m[0] = expf(x0); m[1] = expf(x1); m[2] = expf(x2); m[3] = expf(x3);
 }
 
 // exp(l - max) of the four residual logits, then the Sinkhorn above.
 __device__ __forceinline__ void residual_map(const float* l4, int iters, float m[4]) {
   const float mx = fmaxf(fmaxf(l4[0], l4[1]), fmaxf(l4[2], l4[3]));
   const float mn = fminf(fminf(l4[0], l4[1]), fminf(l4[2], l4[3]));
+  if (mx - mn <= 40.f) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = expf(l4[i] - mx);
-  sinkhorn2(m, iters, mx - mn);
+    for (int i = 0; i < 4; ++i) m[i] = expf(l4[i] - mx);
+    sinkhorn2(m, iters);
+  } else {
+    const float x[4] = {l4[0] - mx, l4[1] - mx, l4[2] - mx, l4[3] - mx};
+    sinkhorn2_log(x, iters, m);
+  }
 }
 
 template <typename T, int TPW, bool WT>

@@ -40,7 +40,7 @@ cudaError_t DevBuf::ensure(size_t want) {
 }
 
 const char* const kProfNames[P_NCAT] = {"gemm", "lm_head", "rmsnorm", "embed", "gdn_prep", "gdn_chunk", "gdn_step",
-                                        "fa_prep", "attention", "mhc", "argmax", "copy"};
+                                        "fa_prep", "attention", "mhc", "argmax", "copy", "gdn_norm"};
 
 Profiler::~Profiler() {
   clear();
@@ -113,18 +113,19 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
   const size_t es = m->esize;
   const int d = c.d;
   const int n_in = m->in_gdn > m->in_fa ? m->in_gdn : m->in_fa;
-  const int o_w = std::max(c.gdn_heads * c.gdn_dv, c.fa_q_heads * c.fa_head_dim);
+  const int Hv = m->gdn_hv;
+  const int o_w = std::max(Hv * c.gdn_dv, c.fa_q_heads * c.fa_head_dim);
   struct Need { DevBuf* b; size_t bytes; } need[] = {
       {&m->h, M * d * es},
       {&m->X, M * c.mhc_streams * d * es},
       {&m->x_in, M * d * es},
       {&m->xn, M * d * es},
       {&m->proj, M * n_in * es},
-      {&m->gq, M * std::max(c.gdn_heads * c.gdn_dk, c.fa_q_heads * c.fa_head_dim) * es},
-      {&m->gk, M * c.gdn_heads * c.gdn_dk * es},
-      {&m->gv, M * c.gdn_heads * c.gdn_dv * es},
-      {&m->gg, M * c.gdn_heads * sizeof(float)},
-      {&m->gb, M * c.gdn_heads * sizeof(float)},
+      {&m->gq, M * std::max(Hv * c.gdn_dk, c.fa_q_heads * c.fa_head_dim) * es},
+      {&m->gk, M * Hv * c.gdn_dk * es},
+      {&m->gv, M * Hv * c.gdn_dv * es},
+      {&m->gg, M * Hv * sizeof(float)},
+      {&m->gb, M * Hv * sizeof(float)},
       {&m->o, M * o_w * es},
       {&m->mix, M * d * es},
       {&m->u, M * d * es},
@@ -134,7 +135,7 @@ static loop_status ensure_workspace(loop_model* m, long M, int B, int Tq, int Tk
       {&m->coeffs, M * 8 * sizeof(float)},
       {&m->rope, (size_t)Tq * (c.rotary_dims / 2) * sizeof(float2)},
       {&m->attn_ws, gqa_scratch_bytes(B, Tq, Tkv_max, c.fa_q_heads, c.fa_kv_heads, c.fa_head_dim, c.dtype)},
-      {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, c.gdn_heads, c.gdn_dk, c.gdn_dv) : 0},
+      {&m->gdn_ws, Tq > 1 ? gdn_workspace_bytes(B, Tq, Hv, c.gdn_dk, c.gdn_dv) : 0},
       {&m->last, (size_t)B * d * es},
   };
   for (auto& n : need) {
@@ -173,16 +174,30 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
           [&] { return rmsnorm(x, nullptr, nullptr, w.attn_norm, m->xn.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (mixer)");
   if (r.kind == 0) {
-    const int H = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
+    // H: heads of the recurrence (the variant's value heads); Hk: key heads
+    const int H = m->gdn_hv, Hk = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
+    const bool variant = cf.gdn_variant == 1;
     gemm_work(M, m->in_gdn, d, EPI_STORE, m->esize, fl, by);
     CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d,
                                 EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "GDN input projection");
-    CK(prof(m, s, P_GDN_PREP, 1, 0, (double)M * (es * (m->in_gdn + 2.0 * H * dk + H * dv) + 8.0 * H),
-            [&] { return lk::gdn_prep(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p,
-                                      (float*)m->gg.p, (float*)m->gb.p, (int)M, H, dk, dv, cf.eps, dt, s); }),
-       "GDN prep");
+    if (variant) {
+      void* conv_state = (char*)c->conv.p + (size_t)r.slot * c->conv_elems * m->esize;
+      // P's q | k | v channels read conv times, the conv inputs before this call, outputs once
+      const double bytes = (double)M * (es * (cf.gdn_conv * (double)m->gdn_ch + 2.0 * H * dk + H * dv) + 16.0 * H) +
+                           4.0 * B * (cf.gdn_conv - 1) * m->gdn_ch * es;
+      CK(prof(m, s, P_GDN_PREP, 2, 0, bytes,
+              [&] { return lk::gdn_conv_prep(m->proj.p, m->in_gdn, w.gdn_conv_w, conv_state, w.gdn_a_bias,
+                                             w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p,
+                                             B, T, Hk, H, dk, dv, cf.gdn_conv, cf.eps, dt, s); }),
+         "GDN conv prep");
+    } else {
+      CK(prof(m, s, P_GDN_PREP, 1, 0, (double)M * (es * (m->in_gdn + 2.0 * H * dk + H * dv) + 8.0 * H),
+              [&] { return lk::gdn_prep(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, m->gq.p, m->gk.p, m->gv.p,
+                                        (float*)m->gg.p, (float*)m->gb.p, (int)M, H, dk, dv, cf.eps, dt, s); }),
+         "GDN prep");
+    }
     float* S = (float*)c->state.p + (size_t)r.slot * c->state_elems;
     const float scale = 1.f / std::sqrt((float)dk);
     // bytes: q, k, v in, o out, gates, and the fp32 state read + written once
@@ -202,6 +217,11 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
                                      dk, dv, scale, dt, s, m->gdn_ws.p); }),
          "GDN chunked scan");
     }
+    if (variant)   // in place: each head's output row is read whole before it is written
+      CK(prof(m, s, P_GDN_NORM, 1, 0, (double)M * H * dv * es * 3.0,
+              [&] { return lk::gdn_gated_norm(m->o.p, (const char*)m->proj.p + (size_t)m->gdn_ch * m->esize,
+                                              m->in_gdn, w.gdn_o_norm, m->o.p, M, H, dv, cf.eps, dt, s); }),
+         "GDN gated output norm");
     gemm_work(M, d, H * dv, EPI_STORE, m->esize, fl, by);
     CK(prof(m, s, P_GEMM, 1, fl, by,
             [&] { return linear(m->o.p, H * dv, w.w_out, nullptr, nullptr, 0, m->mix.p, d, (int)M, d, H * dv, EPI_STORE,
@@ -216,18 +236,26 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
        "FA input projection");
     char* kbase = (char*)c->kv.p + (size_t)r.slot * 2 * c->kv_slab_elems * m->esize;
     char* vbase = kbase + c->kv_slab_elems * m->esize;
-    CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * (Hq + 2 * Hkv) * dh),
-            [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, m->gq.p, kbase, vbase, c->max_tokens, B, T,
-                                     pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt, s,
-                                     (const float2*)m->rope.p); }),
+    // multi-token bf16 queries go raw to the tensor-core attention kernel, which applies
+    // their QK-norm and rotary as it stages them; the prep kernel then writes K and V only
+    const bool fuse_q = dt == BF16 && dh == 256 && T >= 16 && 128 % (Hq / Hkv) == 0 && cf.rotary_dims <= dh / 2;
+    CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * ((fuse_q ? 0 : Hq) + 2 * Hkv) * dh),
+            [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, fuse_q ? nullptr : m->gq.p, kbase, vbase,
+                                     c->max_tokens, B, T, pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt,
+                                     s, (const float2*)m->rope.p); }),
        "QK-norm / rotary / KV write");
     const char* gate = (const char*)m->proj.p + (size_t)Hq * dh * m->esize;
     // causal (query, key) pairs: sum over new tokens of (pos0 + t + 1)
     const double pairs = (double)B * ((double)T * pos0 + (double)T * (T + 1) / 2.0);
     const double attn_bytes = es * ((double)M * Hq * dh * 3.0 + (double)B * Hkv * (pos0 + T) * dh * 2.0);
+    const QNorm qn{w.q_norm, cf.rotary_dims, cf.rope_base, cf.eps, (const float2*)m->rope.p, pos0};
     CK(prof(m, s, P_ATTN, gqa_launches(B, T, pos0 + T, Hq, Hkv, dh, dt, m->attn_ws.p != nullptr), 4.0 * Hq * dh * pairs, attn_bytes,
-            [&] { return lk::gqa_attn(m->gq.p, Hq * dh, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B, T,
-                                      pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s); }),
+            [&] {
+              return fuse_q ? lk::gqa_attn(m->proj.p, m->in_fa, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B,
+                                           T, pos0 + T, pos0, Hq, Hkv, dh, 1, nullptr, dt, s, &qn)
+                            : lk::gqa_attn(m->gq.p, Hq * dh, kbase, vbase, c->max_tokens, gate, m->in_fa, m->o.p, B, T,
+                                           pos0 + T, pos0, Hq, Hkv, dh, 1, m->attn_ws.p, dt, s);
+            }),
        "GQA attention");
     gemm_work(M, d, Hq * dh, EPI_STORE, m->esize, fl, by);
     CK(prof(m, s, P_GEMM, 1, fl, by,

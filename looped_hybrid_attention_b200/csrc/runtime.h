@@ -37,7 +37,7 @@ struct Profiler {
   void clear();
 };
 enum ProfCat { P_GEMM, P_LMHEAD, P_RMSNORM, P_EMBED, P_GDN_PREP, P_GDN_CHUNK, P_GDN_STEP, P_FA_PREP, P_ATTN, P_MHC,
-               P_ARGMAX, P_COPY, P_NCAT };
+               P_ARGMAX, P_COPY, P_GDN_NORM, P_NCAT };
 extern const char* const kProfNames[P_NCAT];
 
 struct loop_model {
@@ -54,6 +54,7 @@ struct loop_model {
   long ws_tokens = 0;
   DevBuf h, X, x_in, xn, proj, gq, gk, gv, gg, gb, o, mix, u, un, act, F, coeffs, attn_ws, gdn_ws, gemm_ws, rope, last;
   int in_gdn = 0, in_fa = 0;
+  int gdn_hv = 0, gdn_ch = 0;    // GDN value heads; conv channels of the variant (q | k | v)
   Profiler prof;
   DevBuf wrt;                    // [n_layers][8][2d] transposed routing maps (looped layers)
   bool wrt_ready = false;
@@ -67,9 +68,10 @@ struct loop_model {
 struct loop_cache {
   const loop_model* model = nullptr;
   int batch = 0, max_tokens = 0, len = 0;
-  DevBuf kv, state;
+  DevBuf kv, state, conv;
   size_t kv_slab_elems = 0;      // elements of one K (or V) slab
   size_t state_elems = 0;        // floats of one GDN state (all sequences)
+  size_t conv_elems = 0;         // elements of one execution's conv inputs (GDN variant; all sequences)
 };
 
 // Set the thread's error message; returns `st`.

@@ -6,6 +6,10 @@
   python -m looped_hybrid_attention_b200.kernel_bench mhc --T 8192
   python -m looped_hybrid_attention_b200.kernel_bench decode --B 16 --T 32768
   python -m looped_hybrid_attention_b200.kernel_bench group --T 8192   (one full-width layer group in the model flow)
+  python -m looped_hybrid_attention_b200.kernel_bench gdnstep --B 64   (recurrent GDN step, 16 heads x 128)
+  python -m looped_hybrid_attention_b200.kernel_bench rmsnorm --M 8192 (d 4096, with the residual sum)
+  python -m looped_hybrid_attention_b200.kernel_bench gdnprep --M 8192 (GDN input preparation, 16 heads)
+  python -m looped_hybrid_attention_b200.kernel_bench faprep --T 8192  (QK-norm, rotary, K/V slab write)
 
 Inputs are random bf16 tensors created on the device (larger than L2 at the default
 sizes); the printed rate uses the same algorithmic flop/byte counts as bench.py.
@@ -35,7 +39,8 @@ def timed(fn, warmup, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemm", "gdn", "attn", "decode", "mhc", "group"])
+    ap.add_argument("op", choices=["gemm", "gdn", "attn", "decode", "mhc", "group", "gdnstep", "rmsnorm", "gdnprep",
+                                   "faprep"])
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
@@ -97,6 +102,46 @@ def main():
         ms = timed(lambda: L.gqa_attn(q, Hq * dh, K, V, T, gate, Hq * dh, out, B, 1, T, T - 1, Hq, Hkv, dh, True, ws),
                    a.warmup, a.iters)
         res.update(shape=[B, T, Hq, Hkv, dh], ms=ms, gbs=B * Hkv * T * dh * 2 * 2 / ms / 1e6)
+    elif a.op == "gdnstep":
+        B, H, dk = a.B, a.H, 128
+        q = torch.nn.functional.normalize(torch.randn(B, H, dk, device=dev, generator=g), dim=-1).to(bf)
+        k = torch.nn.functional.normalize(torch.randn(B, H, dk, device=dev, generator=g), dim=-1).to(bf)
+        v = r(B, H, dk)
+        gg = -torch.nn.functional.softplus(torch.randn(B, H, device=dev, generator=g))
+        beta = torch.sigmoid(torch.randn(B, H, device=dev, generator=g))
+        S = 0.1 * torch.randn(B, H, dk, dk, device=dev, generator=g)
+        out = torch.empty_like(v)
+        ms = timed(lambda: L.gdn_step(q, k, v, gg, beta, S, out, dk ** -0.5), a.warmup, a.iters)
+        byts = 8.0 * B * H * dk * dk + B * H * (4 * dk * 2 + 8)
+        res.update(shape=[B, H, dk], ms=ms, gbs=byts / ms / 1e6)
+    elif a.op == "rmsnorm":
+        M, d = a.M, 4096
+        x, rr, w = r(M, d), r(M, d), r(d)
+        y, sm = torch.empty_like(x), torch.empty_like(x)
+        ms = timed(lambda: L.rmsnorm(x, w, y, 1e-6, r=rr, sum_out=sm), a.warmup, a.iters)
+        res.update(shape=[M, d], ms=ms, gbs=2.0 * 4 * M * d / ms / 1e6)
+    elif a.op == "gdnprep":
+        M, H, dk = a.M, a.H, 128
+        n_in = 3 * H * dk + 2 * H
+        P = r(M, n_in)
+        ab, bb = torch.zeros(H, device=dev), torch.zeros(H, device=dev)
+        q = torch.empty((M, H, dk), device=dev, dtype=bf)
+        k, v = torch.empty_like(q), torch.empty_like(q)
+        gg, beta = torch.empty((M, H), device=dev), torch.empty((M, H), device=dev)
+        ms = timed(lambda: L.gdn_prep(P, ab, bb, q, k, v, gg, beta, H, dk, dk, 1e-6), a.warmup, a.iters)
+        res.update(shape=[M, H, dk], ms=ms, gbs=(2.0 * M * n_in + 2.0 * 3 * M * H * dk + 8.0 * M * H) / ms / 1e6)
+    elif a.op == "faprep":
+        T, Hq, Hkv, dh = a.T, 16, 4, 256
+        P = r(T, 2 * Hq * dh + 2 * Hkv * dh)
+        qn, kn = r(dh), r(dh)
+        qo = torch.empty((T, Hq, dh), device=dev, dtype=bf)
+        K, V = torch.empty((1, Hkv, T, dh), device=dev, dtype=bf), torch.empty((1, Hkv, T, dh), device=dev, dtype=bf)
+        ms = timed(lambda: L.fa_prep(P, qn, kn, qo, K, V, T, 1, T, 0, Hq, Hkv, dh, 64, 10000.0, 1e-6),
+                   a.warmup, a.iters)
+        ms_kv = timed(lambda: L.fa_prep(P, qn, kn, None, K, V, T, 1, T, 0, Hq, Hkv, dh, 64, 10000.0, 1e-6),
+                      a.warmup, a.iters)
+        res.update(shape=[T, Hq, Hkv, dh], ms=ms, gbs=2.0 * T * (Hq + 2 * Hkv) * dh * 2 / ms / 1e6,
+                   kv_only_ms=ms_kv, kv_only_gbs=2.0 * T * (2 * Hkv) * dh * 2 / ms_kv / 1e6)
     elif a.op == "group":
         import synth
         shape = synth.GROUP
