@@ -208,6 +208,16 @@ loop_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
                           void* stream);
 size_t loop_gdn_workspace_bytes(int B, int T, int H, int dk, int dv);
 
+/* The GDN input projection with gdn_prep fused into its epilogue: the product x W_in^T
+ * (x [M, d] row stride ldx, W_in [2*H*dk + H*dv + 2*H, d]) is never stored; each row's
+ * q, k heads are L2-normalised from the fp32 accumulators and written with v, g and beta
+ * exactly as gdn_prep writes them.  Built for the prefill shapes only: bf16, M > 128,
+ * dk = dv = 128, H even and <= 16, 16-byte aligned x, W_in, q, k, v (LOOP_ERR_UNSUPPORTED
+ * otherwise: use loop_linear + gdn_prep). */
+loop_status gdn_in_proj(const void* x, int ldx, const void* w_in, const float* a_bias,
+                        const float* b_bias, void* q, void* k, void* v, float* g, float* beta,
+                        int M, int d, int H, int dk, int dv, float eps, int dtype, void* stream);
+
 /* GDN variant input preparation ("原地套圈" investigation §01, backbone qwen3_5_text): from
  * P [B*T, ld_p] (row blocks q | k (Hk heads) | v | z (Hv heads) | a | b (Hv)): the q | k | v
  * channels c pass through a causal depthwise conv and SiLU,

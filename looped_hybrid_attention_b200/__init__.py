@@ -82,6 +82,7 @@ _SIGS = {
     "gdn_chunk_fwd": ([_P] * 7 + [_I] * 6 + [_F, _P, _I, _P], _I),
     "loop_gdn_workspace_bytes": ([_I] * 5, _Z),
     "gdn_step": ([_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
+    "gdn_in_proj": ([_P, _I, _P, _P, _P, _P, _P, _P, _P, _P] + [_I] * 5 + [_F, _I, _P], _I),
     "gdn_conv_prep": ([_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P] + [_I] * 7 + [_F, _I, _P], _I),
     "gdn_gated_norm": ([_P, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P], _I),
     "gdn_prep": ([_P, _I] + [_P] * 7 + [_I] * 4 + [_F, _I, _P], _I),
@@ -319,6 +320,13 @@ def gdn_prep(P, a_bias, b_bias, q, k, v, g, beta, H, dk, dv, eps, stream=None):
     M = P.shape[0]
     check(_lib.gdn_prep(ptr(P), P.stride(0), ptr(a_bias), ptr(b_bias), ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta),
                         M, H, dk, dv, eps, dtype_code(P), _stream(stream)), "gdn_prep")
+
+
+def gdn_in_proj(x, w_in, a_bias, b_bias, q, k, v, g, beta, H, dk, dv, eps, stream=None):
+    """GDN input projection with the preparation (L2 norms, gates) in its epilogue."""
+    M, d = x.shape
+    check(_lib.gdn_in_proj(ptr(x), x.stride(0), ptr(w_in), ptr(a_bias), ptr(b_bias), ptr(q), ptr(k), ptr(v), ptr(g),
+                           ptr(beta), M, d, H, dk, dv, eps, dtype_code(x), _stream(stream)), "gdn_in_proj")
 
 
 def gdn_conv_prep(P, conv_w, conv_state, a_bias, b_bias, q, k, v, g, beta, B, T, Hk, Hv, dk, dv, eps, conv=4,

@@ -330,6 +330,20 @@ loop_status gdn_gated_norm(const void* o, const void* z, int ld_z, const void* w
   return launched(lk::gdn_gated_norm(o, z, ld_z, w, y, M, H, dv, eps, dtype, S(stream)), "gdn_gated_norm");
 }
 
+loop_status gdn_in_proj(const void* x, int ldx, const void* w_in, const float* a_bias, const float* b_bias, void* q,
+                        void* k, void* v, float* g, float* beta, int M, int d, int H, int dk, int dv, float eps,
+                        int dtype, void* stream) {
+  REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");
+  REQUIRE(M >= 0 && d > 0 && H > 0, LOOP_ERR_INVALID_ARG, "bad size");
+  if (M == 0) return LOOP_OK;
+  REQUIRE(x && w_in && a_bias && b_bias && q && k && v && g && beta, LOOP_ERR_INVALID_ARG, "NULL argument");
+  REQUIRE(ldx >= d, LOOP_ERR_SHAPE, "ldx < d");
+  REQUIRE(dtype == LOOP_BF16 && M > 128 && dk == 128 && dv == 128 && H % 2 == 0 && H <= 16 && d % 8 == 0,
+          LOOP_ERR_UNSUPPORTED, "built for bf16, M > 128, dk = dv = 128, even H <= 16, d a multiple of 8");
+  const GdnEpi ep{q, k, v, g, beta, a_bias, b_bias, eps, H};
+  return launched(linear_gdn(x, ldx, w_in, M, d, ep, S(stream)), "gdn_in_proj");
+}
+
 loop_status gdn_prep(const void* P, int ld_p, const float* a_bias, const float* b_bias, void* q, void* k, void* v,
                      float* g, float* beta, int M, int H, int dk, int dv, float eps, int dtype, void* stream) {
   REQUIRE(dtype_ok(dtype), LOOP_ERR_INVALID_ARG, "bad dtype");

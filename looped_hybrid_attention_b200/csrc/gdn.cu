@@ -757,28 +757,47 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
   }
   const int mt = w >> 1, nt = w & 1;                         // phases 1-2: 4 x 2 output tiles
   const int r0 = mt * 16 + gq, r1 = r0 + 8, ic = nt * 8 + 2 * tq;
+  // The output of chunk c, O = scale (gamma Q S_c^T + P U), is finished during chunk c + 1
+  // (its P U products interleave with the next chunk's K S^T), so it stays off the chain
+  // of dependent products that carries the state; pending[] holds gamma Q S_c^T.
+  float pend[4] = {0.f, 0.f, 0.f, 0.f};
+  int pend_c = -1;                                           // chunk whose output is pending
+  auto finish_output = [&](int pc) {
+    const uint8_t* pb = smb + (pc % L::NSTAGE) * L::STAGE + L::AW_B + L::Q_B + L::K_B;   // P of chunk pc
+    float cp0[4] = {0.f, 0.f, 0.f, 0.f}, cp1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      uint32_t ap[4], bu[2];
+      ldsm_x4(ap, pb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
+      ldsm_x2_t(bu, Ub + (ks * 16 + (lane & 15)) * UP + nt * 8);
+      mma16816((ks & 1) ? cp1 : cp0, ap, bu);
+    }
+    const int pc0 = pc * C, pn = min(C, T_len - pc0);
+    if (r0 < pn)
+      st_bf2(out + (((long)b * T_len + pc0 + r0) * H + h) * DV + i0 + ic, scale * (pend[0] + cp0[0] + cp1[0]),
+             scale * (pend[1] + cp0[1] + cp1[1]));
+    if (r1 < pn)
+      st_bf2(out + (((long)b * T_len + pc0 + r1) * H + h) * DV + i0 + ic, scale * (pend[2] + cp0[2] + cp1[2]),
+             scale * (pend[3] + cp0[3] + cp1[3]));
+  };
   for (int c = 0; c < n_chunks; ++c) {
     const int bi = c % L::NSTAGE;
     if (!tc::mbar_wait(tc::smem_u32(full + bi), (uint32_t)((c / L::NSTAGE) & 1), abort_flag)) break;
-    // every warp has finished chunk c - 1, so its buffer can take chunk c + 2
+    // every warp has finished chunk c - 1's state update (the state copy below is current)
     __syncthreads();
-    if (tid == 0 && c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
     const uint8_t* base = smb + bi * L::STAGE;
     const uint8_t* Awb = base;                               // swizzled tiles (sw_off)
     const uint8_t* Qb = base + L::AW_B;
     const uint8_t* Kb = base + L::AW_B + L::Q_B;
-    const uint8_t* Pb = base + L::AW_B + L::Q_B + L::K_B;
     const float* Upf = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B);
     const float* Gs = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
-    const int c0 = c * C, n = min(C, T_len - c0);
     const float Glast = Gs[C - 1];
     // decay factors depend on G only: computed while the MMA chain below runs
     const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
     const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]), gl = expf(Glast);
-    // phase 1a: Y = K S^T (S as hi + lo) and Q S^T (hi) share the B operand; the lo term and
-    // the odd k-steps go to separate accumulators (short dependent MMA chains)
-    float cy[4] = {0.f, 0.f, 0.f, 0.f}, cy1[4] = {0.f, 0.f, 0.f, 0.f}, cyl[4] = {0.f, 0.f, 0.f, 0.f};
-    float cq[4] = {0.f, 0.f, 0.f, 0.f}, cq1[4] = {0.f, 0.f, 0.f, 0.f};
+    // phase 1a: Y = K S^T (S as hi + lo) and Q S^T (hi) share the B operand; even and odd
+    // k-steps and the lo terms go to separate accumulators (dependent chains of depth 4)
+    float cy[2][4] = {}, cyl[2][4] = {}, cq[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < DK / 16; ++ks) {
       uint32_t ak[4], aq[4], bs[2], bl[2];
@@ -787,20 +806,22 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
       const int srow = (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8;
       ldsm_x2(bs, Sb + srow);
       ldsm_x2(bl, Sl + srow);
-      mma16816((ks & 1) ? cy1 : cy, ak, bs);
-      mma16816(cyl, ak, bl);
-      mma16816((ks & 1) ? cq1 : cq, aq, bs);
+      mma16816(cy[ks & 1], ak, bs);
+      mma16816(cyl[ks & 1], ak, bl);
+      mma16816(cq[ks & 1], aq, bs);
     }
+    // the previous chunk's output (P U) while those products run
+    if (pend_c >= 0) finish_output(pend_c);
+    float y4[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      cy[e] += cy1[e] + cyl[e];
-      cq[e] += cq1[e];
-    }
-    st_bf2_split(Yh + r0 * UP + ic, Yl + r0 * UP + ic, cy[0], cy[1]);
-    st_bf2_split(Yh + r1 * UP + ic, Yl + r1 * UP + ic, cy[2], cy[3]);
+    for (int e = 0; e < 4; ++e) y4[e] = (cy[0][e] + cy[1][e]) + (cyl[0][e] + cyl[1][e]);
+    st_bf2_split(Yh + r0 * UP + ic, Yl + r0 * UP + ic, y4[0], y4[1]);
+    st_bf2_split(Yh + r1 * UP + ic, Yl + r1 * UP + ic, y4[2], y4[3]);
     __syncthreads();
+    // every warp is done with chunk c - 1's tiles (P included), so its buffer takes chunk c + 2
+    if (tid == 0 && c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
     // phase 1b: W S^T = Aw Y with Aw and Y both as hi + lo (lo x lo dropped)
-    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cw1[4] = {0.f, 0.f, 0.f, 0.f}, cwl[4] = {0.f, 0.f, 0.f, 0.f};
+    float cw[2][4] = {}, cwa[2][4] = {}, cwb[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
       uint32_t ah[4], al[4], yh[2], yl[2];
@@ -808,38 +829,29 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
       ldsm_x4(al, Awb + L::HALF + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
       ldsm_x2_t(yh, Yh + (ks * 16 + (lane & 15)) * UP + nt * 8);
       ldsm_x2_t(yl, Yl + (ks * 16 + (lane & 15)) * UP + nt * 8);
-      mma16816((ks & 1) ? cw1 : cw, ah, yh);
-      mma16816(cwl, ah, yl);
-      mma16816(cwl, al, yh);
+      mma16816(cw[ks & 1], ah, yh);
+      mma16816(cwa[ks & 1], ah, yl);
+      mma16816(cwb[ks & 1], al, yh);
     }
     {
-      const float w00 = cw[0] + cw1[0] + cwl[0], w01 = cw[1] + cw1[1] + cwl[1];
-      const float w10 = cw[2] + cw1[2] + cwl[2], w11 = cw[3] + cw1[3] + cwl[3];
-      const float u00 = Upf[r0 * DVS + ic] - w00, u01 = Upf[r0 * DVS + ic + 1] - w01;
-      const float u10 = Upf[r1 * DVS + ic] - w10, u11 = Upf[r1 * DVS + ic + 1] - w11;
+      float wv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wv[e] = (cw[0][e] + cw[1][e]) + ((cwa[0][e] + cwa[1][e]) + (cwb[0][e] + cwb[1][e]));
+      const float u00 = Upf[r0 * DVS + ic] - wv[0], u01 = Upf[r0 * DVS + ic + 1] - wv[1];
+      const float u10 = Upf[r1 * DVS + ic] - wv[2], u11 = Upf[r1 * DVS + ic + 1] - wv[3];
       st_bf2(Ub + r0 * UP + ic, u00, u01);
       st_bf2(Ub + r1 * UP + ic, u10, u11);
       st_bf2_split(Ueb + r0 * UP + ic, Uel + r0 * UP + ic, u00 * e0, u01 * e0);
       st_bf2_split(Ueb + r1 * UP + ic, Uel + r1 * UP + ic, u10 * e1, u11 * e1);
     }
-    __syncthreads();
-    // phase 2b: P U, then the outputs
-    float cp[4] = {0.f, 0.f, 0.f, 0.f};
+    // gamma Q S_c^T of this chunk, finished with P U during the next one
 #pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      uint32_t ap[4], bu[2];
-      ldsm_x4(ap, Pb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x2_t(bu, Ub + (ks * 16 + (lane & 15)) * UP + nt * 8);
-      mma16816(cp, ap, bu);
+    for (int e = 0; e < 2; ++e) {
+      pend[e] = g0 * (cq[0][e] + cq[1][e]);
+      pend[2 + e] = g1 * (cq[0][2 + e] + cq[1][2 + e]);
     }
-    {
-      if (r0 < n)
-        st_bf2(out + (((long)b * T_len + c0 + r0) * H + h) * DV + i0 + ic, scale * fmaf(g0, cq[0], cp[0]),
-               scale * fmaf(g0, cq[1], cp[1]));
-      if (r1 < n)
-        st_bf2(out + (((long)b * T_len + c0 + r1) * H + h) * DV + i0 + ic, scale * fmaf(g1, cq[2], cp[2]),
-               scale * fmaf(g1, cq[3], cp[3]));
-    }
+    pend_c = c;
+    __syncthreads();
     // phase 3: S <- exp(G_last) S + Ue^T K
 #pragma unroll
     for (int j = 0; j < NT3; ++j)
@@ -877,6 +889,10 @@ __global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant_
       st_bf2_split(Sb + (gq + 8) * KP + col, Sl + (gq + 8) * KP + col, st[j][2], st[j][3]);
     }
   }
+  // the last chunk's output (its tiles and U are still in place: nothing was loaded after
+  // it, and U was published by the barrier before the last state update)
+  // (one decision per warp: the products are warp-collective)
+  if (__all_sync(0xffffffffu, pend_c >= 0 && !*abort_flag)) finish_output(pend_c);
 #pragma unroll
   for (int j = 0; j < NT3; ++j) {
     const int col = (w * NT3 + j) * 8 + 2 * tq;

@@ -78,11 +78,66 @@ __device__ __forceinline__ void arrive_remote(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
+// EPI_GDN: one row's 128 columns of a q or k head from TMEM (4 loads of 32), L2-normalised
+// and stored; v heads copied; the gate tile turned into g and beta.  The TMEM loads are
+// warp-collective: every lane issues them, and only the stores are guarded by the row.
+__device__ __forceinline__ void gdn_epilogue(uint32_t t_row, int row, int n0, int M, const GdnEpi& ep) {
+  const int H = ep.H, qk = 2 * H * 128, vend = qk + H * 128;
+  const bool ok = row < M;
+  if (n0 < vend) {
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {                  // the tile's two heads
+      const int col = n0 + hh * 128;
+      const uint32_t th = t_row + hh * 128;
+      float inv = 1.f;
+      if (col < qk) {
+        float ss = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(th + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
+        }
+        inv = rsqrtf(ss + ep.eps);
+      }
+      __nv_bfloat16* dst;
+      if (col < H * 128) dst = (__nv_bfloat16*)ep.q + ((long)row * H + col / 128) * 128;
+      else if (col < qk) dst = (__nv_bfloat16*)ep.k + ((long)row * H + (col - H * 128) / 128) * 128;
+      else dst = (__nv_bfloat16*)ep.v + ((long)row * H + (col - qk) / 128) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(th + c * 32, r);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv;
+        if (ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) store8(dst + c * 32 + i, v + i);
+        }
+      }
+    }
+  } else {                                            // gates: a (H columns) then b (H columns)
+    uint32_t r[32];
+    tmem_ld32(t_row, r);
+    tmem_wait_ld();
+    for (int j = 0; ok && j < H && j < 16; ++j) {
+      const float a = __uint_as_float(r[j]) + ep.a_bias[j];
+      const float b = __uint_as_float(r[H + j]) + ep.b_bias[j];
+      ep.g[(long)row * H + j] = -(a > 20.f ? a : log1pf(expf(a)));
+      ep.beta[(long)row * H + j] = 1.f / (1.f + expf(-b));
+    }
+  }
+}
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                      const __grid_constant__ CUtensorMap tB2, void* __restrict__ Y, int ldy,
-                     const __nv_bfloat16* R, int ldr, int M, int N, int K, int vec_ok) {
+                     const __nv_bfloat16* R, int ldr, int M, int N, int K, int vec_ok, const GdnEpi ep) {
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;   // output columns per pair tile
   extern __shared__ uint8_t smem_raw[];
   // the same offsets in both CTAs: descriptors and barriers are addressed by offset
@@ -203,8 +258,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       fence_after();
       const int row = m0 + (int)rank * BM + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == EPI_GDN) gdn_epilogue(t_row, row, n0, M, ep);
 #pragma unroll 1
-      for (int c = 0; c < OUT_COLS / 32; ++c) {
+      for (int c = 0; c < (EPI == EPI_GDN ? 0 : OUT_COLS / 32); ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         float v[32];
@@ -275,7 +331,7 @@ done:
 
 template <int EPI>
 static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y,
-                          int ldy, int M, int N, int K, cudaStream_t s) {
+                          int ldy, int M, int N, int K, cudaStream_t s, const GdnEpi& ep = GdnEpi{}) {
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   CUtensorMap tA, tB, tB2;
   if (!make_map(&tA, X, M, K, ldx, BM)) return cudaErrorNotSupported;
@@ -295,7 +351,8 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
   const int esz = EPI == EPI_F32 ? 4 : 2;
   const int vec_ok = ((ldy * esz) % 16 == 0) && (((uintptr_t)Y) % 16 == 0) &&
                      (EPI != EPI_ADD || ((ldr * 2) % 16 == 0 && ((uintptr_t)R) % 16 == 0));
-  kern<<<(unsigned)(2 * pairs), 192, SMEM, s>>>(tA, tB, tB2, Y, ldy, (const __nv_bfloat16*)R, ldr, M, N, K, vec_ok);
+  kern<<<(unsigned)(2 * pairs), 192, SMEM, s>>>(tA, tB, tB2, Y, ldy, (const __nv_bfloat16*)R, ldr, M, N, K, vec_ok,
+                                                 ep);
   return cudaGetLastError();
 }
 
@@ -311,6 +368,15 @@ cudaError_t linear_pair(const void* X, int ldx, const void* W, const void* W2, c
     case EPI_F32: return tc::p2::launch<EPI_F32>(X, ldx, W, W2, R, ldr, Y, ldy, M, N, K, s);
   }
   return cudaErrorNotSupported;
+}
+
+cudaError_t linear_gdn(const void* X, int ldx, const void* W, int M, int K, const GdnEpi& ep, cudaStream_t s) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  if (M <= 128 || ep.H % 2 != 0 || ep.H > 16 || !al16(X) || !al16(W) || (ldx * 2) % 16 || (K * 2) % 16 ||
+      !al16(ep.q) || !al16(ep.k) || !al16(ep.v))
+    return cudaErrorNotSupported;
+  const int N = 3 * ep.H * 128 + 2 * ep.H;
+  return tc::p2::launch<EPI_GDN>(X, ldx, W, nullptr, nullptr, 0, nullptr, 0, M, N, K, s, ep);
 }
 
 }  // namespace lk

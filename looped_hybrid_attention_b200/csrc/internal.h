@@ -7,7 +7,21 @@
 namespace lk {
 
 enum Dtype { F32 = 0, BF16 = 1 };
-enum Epilogue { EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_F32 = 3 };
+enum Epilogue { EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_F32 = 3, EPI_GDN = 4 };
+
+// Outputs of the GDN input projection's fused epilogue (EPI_GDN): q, k L2-normalised per head,
+// v, and the gates g = -softplus(a + a_bias), beta = sigmoid(b + b_bias), from the columns
+// q | k | v | a | b of the product (what gdn_prep computes from the stored projection).
+struct GdnEpi {
+  void *q, *k, *v;          // [M, H, 128] bf16
+  float *g, *beta;          // [M, H] fp32
+  const float *a_bias, *b_bias;
+  float eps;
+  int H;
+};
+// The projection with the GDN preparation in its epilogue (bf16, M > 128, dk = dv = 128,
+// H even); cudaErrorNotSupported otherwise.
+cudaError_t linear_gdn(const void* X, int ldx, const void* W, int M, int K, const GdnEpi& ep, cudaStream_t s);
 enum MhcMode { MHC_OPEN = 0, MHC_MIX = 1, MHC_ROUTE = 2, MHC_MERGE = 3 };
 
 // ldx: row stride of x in elements (0 = d); r, sum_out and y are dense [M, d].

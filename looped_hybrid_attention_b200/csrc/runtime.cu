@@ -177,12 +177,23 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
     // H: heads of the recurrence (the variant's value heads); Hk: key heads
     const int H = m->gdn_hv, Hk = cf.gdn_heads, dk = cf.gdn_dk, dv = cf.gdn_dv;
     const bool variant = cf.gdn_variant == 1;
+    // prefill-sized bf16 batches: the preparation (L2 norms, gates) runs in the projection's
+    // epilogue, so the projection is never stored
+    const bool fused_prep = !variant && dt == BF16 && M > 128 && dk == 128 && dv == 128 && H % 2 == 0 && H <= 16;
     gemm_work(M, m->in_gdn, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
-            [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn, d,
-                                EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
-       "GDN input projection");
-    if (variant) {
+    if (fused_prep) {
+      const GdnEpi ep{m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, w.gdn_a_bias, w.gdn_b_bias,
+                      cf.eps, H};
+      CK(prof(m, s, P_GEMM, 1, fl, by, [&] { return linear_gdn(m->xn.p, d, w.w_in, (int)M, d, ep, s); }),
+         "GDN input projection + preparation");
+    } else {
+      CK(prof(m, s, P_GEMM, 1, fl, by,
+              [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_gdn, (int)M, m->in_gdn,
+                                  d, EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
+         "GDN input projection");
+    }
+    if (fused_prep) {
+    } else if (variant) {
       void* conv_state = (char*)c->conv.p + (size_t)r.slot * c->conv_elems * m->esize;
       // P's q | k | v channels read conv times, the conv inputs before this call, outputs once
       const double bytes = (double)M * (es * (cf.gdn_conv * (double)m->gdn_ch + 2.0 * H * dk + H * dv) + 16.0 * H) +

@@ -81,7 +81,7 @@ def test_variant_tiny_stack_prefill_decode_fp32(cuda):
     every GDN state and conv-input slot against the oracle's cache."""
     import looped_hybrid_attention_b200 as L
     s = VARIANT_TINY
-    w = synth.make_weights(s, seed=11, std=0.05)
+    w = synth.make_weights(s, seed=11)
     W = omodel.Weights(w)
     B, T1, T2 = 2, 60, 2
     ids = synth.uniform_ids((B, T1 + T2 + 3), s.vocab, 11)
