@@ -635,8 +635,8 @@ __global__ void __launch_bounds__(256) gdn_scan_kernel(const T* __restrict__ q, 
 
 
 // ------------------------------------------------------------------ tensor-core sequential pass (bf16)
-// The same recurrence as gdn_scan_kernel with the per-chunk products on the tensor cores
-// (mma.sync m16n8k16, bf16 operands, fp32 accumulation):
+// The bf16 two-pass scan runs its chunk recurrence with the per-chunk products on the tensor
+// cores (mma.sync m16n8k16, bf16 operands, fp32 accumulation):
 //   Y  = K S^T               (64 x 16, K = dk)      A = K (exact),  B = S as bf16 hi + lo
 //   U  = U' - Aw Y           (64 x 16, K = 64)      A = Aw hi + lo, B = Y hi + lo   (W S^T = Aw K S^T)
 //   O  = gamma Q S^T + P U   (64 x 16, K = dk, 64)  A = Q, P; B = S hi, U (output: bf16 operands)
@@ -644,262 +644,332 @@ __global__ void __launch_bounds__(256) gdn_scan_kernel(const T* __restrict__ q, 
 // Every product on the state's path has exact operands or operands carried as two bf16
 // terms (hi + lo, relative error ~2^-17; the lo x lo term is dropped), so the state is
 // updated with fp32-grade accuracy; only the output products use single bf16 operands.
-// The fp32 state lives in registers as the accumulator of the last product; each warp
-// owns dk/64 8-column tiles of the 16 state rows of this CTA.
 __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float x, float y) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x, y);
 }
-// x ~ hi + lo as two bf16 pairs
-__device__ __forceinline__ void st_bf2_split(__nv_bfloat16* hi, __nv_bfloat16* lo, float x, float y) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
-  const float2 f = __bfloat1622float2(h);
-  *reinterpret_cast<__nv_bfloat162*>(hi) = h;
-  *reinterpret_cast<__nv_bfloat162*>(lo) = __floats2bfloat162_rn(x - f.x, y - f.y);
-}
 
-// Shared-memory plan of the tensor-core scan.  A chunk's Aw (hi and lo, [128 rows x 64]),
-// Q, K (64 x dk) and P (64 x 64) arrive by TMA as 64-column pieces of [rows x 128 B] with
-// the 128-byte swizzle (16-byte chunk j of row r stored at j ^ (r & 7)); U' (this CTA's 16
-// columns, fp32) and G (fp32) as plain boxes.  Seven or nine tile loads per chunk,
-// completing on the stage's mbarrier.
+
+// ------------------------------------------------------------------ warp-specialised sequential pass (bf16)
+// The products above split by role, so that the state's chain of dependent
+// products runs on warps of its own and no A fragment is loaded twice:
+//   warps 0-3 (state):  Y = K S^T and U = U' - Aw Y with each warp owning one 16-row m-tile
+//                       of the chunk and both 8-column n-tiles of the CTA's 16 state rows;
+//                       S <- exp(G_C) S + (eU)^T K with each warp owning a quarter of the dk
+//                       columns.  State-path operands as hi + lo bf16 pairs, as above.
+//   warps 4-7 (output): O = scale (gamma Q S_c^T + P U) for the same m-tiles (bf16 hi
+//                       operands), at most one chunk behind the state warps.
+//   warp 8 (producer):  the chunk's tiles by TMA into a 3-stage ring.
+// Hand-offs: mbarriers full[s] (the stage's tiles landed), empty[s] (the 8 compute warps
+// are done with the stage), go[c % 2] (U of chunk c and the state it started from are in
+// shared memory), done (the output warps finished a chunk: its U buffer and the state copy
+// it read may be reused); named barrier 1 among the 128 state threads.  Shared-memory
+// addresses of the fragments are fixed per lane and computed once.
 template <int DK, int DV>
-struct ScanTc {
+struct ScanWs {
   static constexpr int C = GDN_C, DVS = 16, KP = DK + 8, UP = DVS + 8;
-  static constexpr int HALF = C * 128;                       // one 64-column piece of 64 rows, 8 KB
+  static constexpr int HALF = C * 128;
   static constexpr int AW_B = 2 * HALF, Q_B = (DK / 64) * HALF, K_B = Q_B, P_B = HALF, UPF_B = C * DVS * 4,
                        G_B = C * 4;
-  static constexpr int TX = AW_B + Q_B + K_B + P_B + UPF_B + G_B;    // bytes per chunk
-  static constexpr int STAGE = (TX + 1023) / 1024 * 1024;            // swizzled tiles: 1024-byte aligned
-  static constexpr int SB_B = DVS * KP * 2, UB_B = C * UP * 2;
-  static constexpr int NSTAGE = 3;                           // chunks in flight: two ahead of the one in use
-  // state hi, lo; U; exp(G_last - G) U hi, lo; Y hi, lo
-  static constexpr int BAR_OFF = NSTAGE * STAGE + 2 * SB_B + 5 * UB_B;   // NSTAGE mbarriers, then an abort flag
-  static constexpr size_t BYTES = (size_t)BAR_OFF + 8 * NSTAGE + 16 + 1024;   // + alignment slack
+  static constexpr int TX = AW_B + Q_B + K_B + P_B + UPF_B + G_B;
+  static constexpr int STAGE = (TX + 1023) / 1024 * 1024;
+  static constexpr int NSTAGE = 3;
+  static constexpr int S_B = DVS * KP * 2, U_B = C * UP * 2;
+  // state copies [2 buffers][hi, lo]; U for the output [2 buffers]; (eU) hi, lo; Y hi, lo
+  static constexpr int OFF_S = NSTAGE * STAGE, OFF_U = OFF_S + 4 * S_B, OFF_UE = OFF_U + 2 * U_B,
+                       OFF_Y = OFF_UE + 2 * U_B, BAR_OFF = OFF_Y + 2 * U_B;
+  static constexpr int N_BARS = 2 * NSTAGE + 3;                 // full[3], empty[3], go[2], done
+  static constexpr size_t BYTES = (size_t)BAR_OFF + 8 * N_BARS + 16 + 1024;
   static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
+  static_assert(BYTES <= 232448, "shared memory per CTA");
 };
 
-// Byte offset of bf16 element (row, col) (col a multiple of 8) in a tile stored as 64-column
-// pieces of [GDN_C rows x 128 B] with the 128-byte swizzle (rows < 64 per piece).
-__device__ __forceinline__ uint32_t sw_off(int row, int col) {
-  return (uint32_t)((col >> 6) * (GDN_C * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+// Shared-memory accesses by address (explicit shared-window loads and stores).
+__device__ __forceinline__ float lds_f(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_bf2(uint32_t a, float x, float y) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(pack_bf2(x, y)) : "memory");
+}
+__device__ __forceinline__ void sts_bf2_split(uint32_t hi, uint32_t lo, float x, float y) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 f = __bfloat1622float2(h);
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(hi), "r"(*reinterpret_cast<const uint32_t*>(&h)) : "memory");
+  sts_bf2(lo, x - f.x, y - f.y);
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap mA,
-                                                          const __grid_constant__ CUtensorMap mP,
-                                                          const __grid_constant__ CUtensorMap mU,
-                                                          const __grid_constant__ CUtensorMap mG,
-                                                          const __grid_constant__ CUtensorMap mQ,
-                                                          const __grid_constant__ CUtensorMap mK, float* __restrict__ state,
-                                                          __nv_bfloat16* __restrict__ out, int T_len, int H,
-                                                          int n_chunks, float scale) {
-  using L = ScanTc<DK, DV>;
+__global__ void __launch_bounds__(288, 1) gdn_scan_ws_kernel(const __grid_constant__ CUtensorMap mA,
+                                                             const __grid_constant__ CUtensorMap mP,
+                                                             const __grid_constant__ CUtensorMap mU,
+                                                             const __grid_constant__ CUtensorMap mG,
+                                                             const __grid_constant__ CUtensorMap mQ,
+                                                             const __grid_constant__ CUtensorMap mK,
+                                                             float* __restrict__ state, __nv_bfloat16* __restrict__ out,
+                                                             int T_len, int H, int n_chunks, float scale) {
+  using L = ScanWs<DK, DV>;
   constexpr int C = L::C, DVS = L::DVS, KP = L::KP, UP = L::UP;
-  constexpr int NT3 = DK / 64;                               // state column tiles per warp
-  extern __shared__ __align__(16) uint8_t smb_raw[];
-  uint8_t* smb = (uint8_t*)(((uintptr_t)smb_raw + 1023) & ~(uintptr_t)1023);
-  __nv_bfloat16* Sb = (__nv_bfloat16*)(smb + L::NSTAGE * L::STAGE);  // [DVS][KP] state slice, bf16 hi part
-  __nv_bfloat16* Sl = Sb + DVS * KP;                         // ... and lo part
-  __nv_bfloat16* Ub = Sl + DVS * KP;                         // [C][UP] U (bf16, output product)
-  __nv_bfloat16* Ueb = Ub + C * UP;                          // [C][UP] exp(G_last - G_s) U, hi
-  __nv_bfloat16* Uel = Ueb + C * UP;                         // ... lo
-  __nv_bfloat16* Yh = Uel + C * UP;                          // [C][UP] Y = K S^T, hi
-  __nv_bfloat16* Yl = Yh + C * UP;                           // ... lo
-  uint64_t* full = reinterpret_cast<uint64_t*>(smb + L::BAR_OFF);   // a chunk's tiles landed, per stage
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + L::NSTAGE);
+  extern __shared__ __align__(16) uint8_t smw_raw[];
+  uint8_t* smb = (uint8_t*)(((uintptr_t)smw_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = tc::smem_u32(smb);
+  const uint32_t bar0 = sbase + L::BAR_OFF;
+  auto full = [&](int i) { return bar0 + 8u * i; };
+  auto empty = [&](int i) { return bar0 + 8u * (L::NSTAGE + i); };
+  auto go = [&](int i) { return bar0 + 8u * (2 * L::NSTAGE + i); };
+  const uint32_t done = bar0 + 8u * (2 * L::NSTAGE + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smb + L::BAR_OFF + 8 * L::N_BARS);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int i0 = blockIdx.x * DVS, h = blockIdx.y, b = blockIdx.z;
   if (tid == 0) {
-    for (int i = 0; i < L::NSTAGE; ++i) tc::mbar_init(tc::smem_u32(full + i), 1);
+    for (int i = 0; i < L::NSTAGE; ++i) {
+      tc::mbar_init(full(i), 1);
+      tc::mbar_init(empty(i), 8);                              // one arrival per compute warp
+    }
+    tc::mbar_init(go(0), 4);
+    tc::mbar_init(go(1), 4);
+    tc::mbar_init(done, 4);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mA) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mQ) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mK) : "memory");
   }
-  const int i0 = blockIdx.x * DVS, h = blockIdx.y, b = blockIdx.z;
   float* Sg = state + (((long)b * H + h) * DV + i0) * DK;
+  // byte offsets (from sbase) of the shared arrays
+  auto s_copy = [&](int buf, int lo) { return (uint32_t)(L::OFF_S + (2 * buf + lo) * L::S_B); };
+  const uint32_t u_out0 = L::OFF_U, ueh = L::OFF_UE, uel = L::OFF_UE + L::U_B, yh = L::OFF_Y, yl = L::OFF_Y + L::U_B;
+  auto stage_off = [&](int c) { return (uint32_t)((c % L::NSTAGE) * L::STAGE); };
+  // per-lane fragment offsets
+  const int mt = w & 3;                                        // the m-tile of a state or output warp
+  uint32_t a_off[4];                                           // A fragments of a swizzled 64-row piece
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    a_off[kk] = (uint32_t)((mt * 16 + (lane & 15)) * 128 + ((((2 * kk + (lane >> 4)) ^ (lane & 7)) & 7) << 4));
+  const uint32_t b_s = (uint32_t)(((lane & 7) + (lane >> 4) * 8) * KP * 2 + ((lane >> 3) & 1) * 16);  // state copy
+  const uint32_t b_y = (uint32_t)((lane & 15) * UP * 2 + (lane >> 4) * 16);                            // [C][UP], trans
+  const uint32_t a_ue = (uint32_t)((((lane >> 4) * 8) + (lane & 7)) * UP * 2 + ((lane >> 3) & 1) * 16);  // (eU)^T
+  const int r0 = mt * 16 + gq, r1 = r0 + 8;
 
-  float st[NT3][4];
-#pragma unroll
-  for (int j = 0; j < NT3; ++j) {
-    const int col = (w * NT3 + j) * 8 + 2 * tq;
-    st[j][0] = Sg[gq * DK + col];
-    st[j][1] = Sg[gq * DK + col + 1];
-    st[j][2] = Sg[(gq + 8) * DK + col];
-    st[j][3] = Sg[(gq + 8) * DK + col + 1];
-    st_bf2_split(Sb + gq * KP + col, Sl + gq * KP + col, st[j][0], st[j][1]);
-    st_bf2_split(Sb + (gq + 8) * KP + col, Sl + (gq + 8) * KP + col, st[j][2], st[j][3]);
-  }
+  __syncthreads();                                             // barriers initialised
 
-  // one thread: the chunk's tiles (rows past the sequence end read as zeros)
-  auto issue = [&](int c, int bi) {
-    uint8_t* base = smb + bi * L::STAGE;
-    const int blk = ((b * H + h) * n_chunks + c);
-    const uint32_t fb = tc::smem_u32(full + bi);
-    tc::fence_proxy_async();                                 // earlier generic reads of this stage first
-    tc::mbar_expect_tx(fb, (uint32_t)L::TX);
-    tc::tma_load_3d(tc::smem_u32(base), &mA, fb, 0, 0, blk);
+  if (w == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mA) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mQ) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mK) : "memory");
+      for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % L::NSTAGE;
+        if (c >= L::NSTAGE && !tc::mbar_wait(empty(st), (uint32_t)((c / L::NSTAGE - 1) & 1), abort_flag)) break;
+        tc::fence_proxy_async();                               // the consumers' reads before the new tiles
+        const uint32_t base = sbase + stage_off(c);
+        const int blk = (b * H + h) * n_chunks + c;
+        const uint32_t fb = full(st);
+        tc::mbar_expect_tx(fb, (uint32_t)L::TX);
+        tc::tma_load_3d(base, &mA, fb, 0, 0, blk);
 #pragma unroll
-    for (int hf = 0; hf < DK / 64; ++hf) {
-      tc::tma_load_4d(tc::smem_u32(base + L::AW_B + hf * L::HALF), &mQ, fb, hf * 64, h, c * C, b);
-      tc::tma_load_4d(tc::smem_u32(base + L::AW_B + L::Q_B + hf * L::HALF), &mK, fb, hf * 64, h, c * C, b);
-    }
-    const int off_p = L::AW_B + L::Q_B + L::K_B;
-    tc::tma_load_3d(tc::smem_u32(base + off_p), &mP, fb, 0, 0, blk);
-    tc::tma_load_3d(tc::smem_u32(base + off_p + L::P_B), &mU, fb, i0, 0, blk);
-    tc::tma_load_2d(tc::smem_u32(base + off_p + L::P_B + L::UPF_B), &mG, fb, 0, blk);
-  };
-
-  __syncthreads();                                           // barriers initialised
-  if (tid == 0) {
-    issue(0, 0);
-    if (n_chunks > 1) issue(1, 1);
-  }
-  const int mt = w >> 1, nt = w & 1;                         // phases 1-2: 4 x 2 output tiles
-  const int r0 = mt * 16 + gq, r1 = r0 + 8, ic = nt * 8 + 2 * tq;
-  // The output of chunk c, O = scale (gamma Q S_c^T + P U), is finished during chunk c + 1
-  // (its P U products interleave with the next chunk's K S^T), so it stays off the chain
-  // of dependent products that carries the state; pending[] holds gamma Q S_c^T.
-  float pend[4] = {0.f, 0.f, 0.f, 0.f};
-  int pend_c = -1;                                           // chunk whose output is pending
-  auto finish_output = [&](int pc) {
-    const uint8_t* pb = smb + (pc % L::NSTAGE) * L::STAGE + L::AW_B + L::Q_B + L::K_B;   // P of chunk pc
-    float cp0[4] = {0.f, 0.f, 0.f, 0.f}, cp1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      uint32_t ap[4], bu[2];
-      ldsm_x4(ap, pb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x2_t(bu, Ub + (ks * 16 + (lane & 15)) * UP + nt * 8);
-      mma16816((ks & 1) ? cp1 : cp0, ap, bu);
-    }
-    const int pc0 = pc * C, pn = min(C, T_len - pc0);
-    if (r0 < pn)
-      st_bf2(out + (((long)b * T_len + pc0 + r0) * H + h) * DV + i0 + ic, scale * (pend[0] + cp0[0] + cp1[0]),
-             scale * (pend[1] + cp0[1] + cp1[1]));
-    if (r1 < pn)
-      st_bf2(out + (((long)b * T_len + pc0 + r1) * H + h) * DV + i0 + ic, scale * (pend[2] + cp0[2] + cp1[2]),
-             scale * (pend[3] + cp0[3] + cp1[3]));
-  };
-  for (int c = 0; c < n_chunks; ++c) {
-    const int bi = c % L::NSTAGE;
-    if (!tc::mbar_wait(tc::smem_u32(full + bi), (uint32_t)((c / L::NSTAGE) & 1), abort_flag)) break;
-    // every warp has finished chunk c - 1's state update (the state copy below is current)
-    __syncthreads();
-    const uint8_t* base = smb + bi * L::STAGE;
-    const uint8_t* Awb = base;                               // swizzled tiles (sw_off)
-    const uint8_t* Qb = base + L::AW_B;
-    const uint8_t* Kb = base + L::AW_B + L::Q_B;
-    const float* Upf = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B);
-    const float* Gs = (const float*)(base + L::AW_B + L::Q_B + L::K_B + L::P_B + L::UPF_B);
-    const float Glast = Gs[C - 1];
-    // decay factors depend on G only: computed while the MMA chain below runs
-    const float e0 = expf(Glast - Gs[r0]), e1 = expf(Glast - Gs[r1]);
-    const float g0 = expf(Gs[r0]), g1 = expf(Gs[r1]), gl = expf(Glast);
-    // phase 1a: Y = K S^T (S as hi + lo) and Q S^T (hi) share the B operand; even and odd
-    // k-steps and the lo terms go to separate accumulators (dependent chains of depth 4)
-    float cy[2][4] = {}, cyl[2][4] = {}, cq[2][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < DK / 16; ++ks) {
-      uint32_t ak[4], aq[4], bs[2], bl[2];
-      ldsm_x4(ak, Kb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x4(aq, Qb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      const int srow = (nt * 8 + (lane & 7)) * KP + ks * 16 + ((lane >> 3) & 1) * 8;
-      ldsm_x2(bs, Sb + srow);
-      ldsm_x2(bl, Sl + srow);
-      mma16816(cy[ks & 1], ak, bs);
-      mma16816(cyl[ks & 1], ak, bl);
-      mma16816(cq[ks & 1], aq, bs);
-    }
-    // the previous chunk's output (P U) while those products run
-    if (pend_c >= 0) finish_output(pend_c);
-    float y4[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y4[e] = (cy[0][e] + cy[1][e]) + (cyl[0][e] + cyl[1][e]);
-    st_bf2_split(Yh + r0 * UP + ic, Yl + r0 * UP + ic, y4[0], y4[1]);
-    st_bf2_split(Yh + r1 * UP + ic, Yl + r1 * UP + ic, y4[2], y4[3]);
-    __syncthreads();
-    // every warp is done with chunk c - 1's tiles (P included), so its buffer takes chunk c + 2
-    if (tid == 0 && c + 2 < n_chunks) issue(c + 2, (c + 2) % L::NSTAGE);
-    // phase 1b: W S^T = Aw Y with Aw and Y both as hi + lo (lo x lo dropped)
-    float cw[2][4] = {}, cwa[2][4] = {}, cwb[2][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      uint32_t ah[4], al[4], yh[2], yl[2];
-      ldsm_x4(ah, Awb + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x4(al, Awb + L::HALF + sw_off(mt * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8));
-      ldsm_x2_t(yh, Yh + (ks * 16 + (lane & 15)) * UP + nt * 8);
-      ldsm_x2_t(yl, Yl + (ks * 16 + (lane & 15)) * UP + nt * 8);
-      mma16816(cw[ks & 1], ah, yh);
-      mma16816(cwa[ks & 1], ah, yl);
-      mma16816(cwb[ks & 1], al, yh);
-    }
-    {
-      float wv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) wv[e] = (cw[0][e] + cw[1][e]) + ((cwa[0][e] + cwa[1][e]) + (cwb[0][e] + cwb[1][e]));
-      const float u00 = Upf[r0 * DVS + ic] - wv[0], u01 = Upf[r0 * DVS + ic + 1] - wv[1];
-      const float u10 = Upf[r1 * DVS + ic] - wv[2], u11 = Upf[r1 * DVS + ic + 1] - wv[3];
-      st_bf2(Ub + r0 * UP + ic, u00, u01);
-      st_bf2(Ub + r1 * UP + ic, u10, u11);
-      st_bf2_split(Ueb + r0 * UP + ic, Uel + r0 * UP + ic, u00 * e0, u01 * e0);
-      st_bf2_split(Ueb + r1 * UP + ic, Uel + r1 * UP + ic, u10 * e1, u11 * e1);
-    }
-    // gamma Q S_c^T of this chunk, finished with P U during the next one
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      pend[e] = g0 * (cq[0][e] + cq[1][e]);
-      pend[2 + e] = g1 * (cq[0][2 + e] + cq[1][2 + e]);
-    }
-    pend_c = c;
-    __syncthreads();
-    // phase 3: S <- exp(G_last) S + Ue^T K
-#pragma unroll
-    for (int j = 0; j < NT3; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st[j][e] *= gl;
-    // the odd k-steps and the lo terms accumulate separately (independent MMA chains of
-    // depth 2) and are added at the end
-    float st1[NT3][4], sl0[NT3][4], sl1[NT3][4];
-#pragma unroll
-    for (int j = 0; j < NT3; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st1[j][e] = sl0[j][e] = sl1[j][e] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      uint32_t au[4], al[4];
-      const int urow = (ks * 16 + (lane >> 4) * 8 + (lane & 7)) * UP + ((lane >> 3) & 1) * 8;
-      ldsm_x4_t(au, Ueb + urow);
-      ldsm_x4_t(al, Uel + urow);
-#pragma unroll
-      for (int j = 0; j < NT3; ++j) {
-        uint32_t bk[2];
-        ldsm_x2_t(bk, Kb + sw_off(ks * 16 + (lane & 15), (w * NT3 + j) * 8));
-        mma16816((ks & 1) ? st1[j] : st[j], au, bk);
-        mma16816((ks & 1) ? sl1[j] : sl0[j], al, bk);
+        for (int hf = 0; hf < DK / 64; ++hf) {
+          tc::tma_load_4d(base + L::AW_B + hf * L::HALF, &mQ, fb, hf * 64, h, c * C, b);
+          tc::tma_load_4d(base + L::AW_B + L::Q_B + hf * L::HALF, &mK, fb, hf * 64, h, c * C, b);
+        }
+        const uint32_t off_p = L::AW_B + L::Q_B + L::K_B;
+        tc::tma_load_3d(base + off_p, &mP, fb, 0, 0, blk);
+        tc::tma_load_3d(base + off_p + L::P_B, &mU, fb, i0, 0, blk);
+        tc::tma_load_2d(base + off_p + L::P_B + L::UPF_B, &mG, fb, 0, blk);
       }
     }
+  } else if (w < 4) {
+    // ---------------------------------------------------------------- state warps
+    constexpr int NT = DK / 32;                                // 8-column state tiles per warp
+    const int cb = w * NT;                                     // first state tile of this warp
+    // B fragments of K (trans) for the tile pairs (cb, cb+1), (cb+2, cb+3), ...
+    uint32_t b_k[NT / 2];
 #pragma unroll
-    for (int j = 0; j < NT3; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st[j][e] += st1[j][e] + (sl0[j][e] + sl1[j][e]);
-#pragma unroll
-    for (int j = 0; j < NT3; ++j) {
-      const int col = (w * NT3 + j) * 8 + 2 * tq;
-      st_bf2_split(Sb + gq * KP + col, Sl + gq * KP + col, st[j][0], st[j][1]);
-      st_bf2_split(Sb + (gq + 8) * KP + col, Sl + (gq + 8) * KP + col, st[j][2], st[j][3]);
+    for (int p = 0; p < NT / 2; ++p) {
+      const int col = (cb + 2 * p + (lane >> 4)) * 8;
+      b_k[p] = (uint32_t)((col >> 6) * L::HALF + (lane & 15) * 128 + ((((col & 63) >> 3) ^ (lane & 7)) << 4));
     }
-  }
-  // the last chunk's output (its tiles and U are still in place: nothing was loaded after
-  // it, and U was published by the barrier before the last state update)
-  // (one decision per warp: the products are warp-collective)
-  if (__all_sync(0xffffffffu, pend_c >= 0 && !*abort_flag)) finish_output(pend_c);
+    float st[NT][4];
 #pragma unroll
-  for (int j = 0; j < NT3; ++j) {
-    const int col = (w * NT3 + j) * 8 + 2 * tq;
-    Sg[gq * DK + col] = st[j][0];
-    Sg[gq * DK + col + 1] = st[j][1];
-    Sg[(gq + 8) * DK + col] = st[j][2];
-    Sg[(gq + 8) * DK + col + 1] = st[j][3];
+    for (int j = 0; j < NT; ++j) {
+      const int col = (cb + j) * 8 + 2 * tq;
+      st[j][0] = Sg[gq * DK + col];
+      st[j][1] = Sg[gq * DK + col + 1];
+      st[j][2] = Sg[(gq + 8) * DK + col];
+      st[j][3] = Sg[(gq + 8) * DK + col + 1];
+      const uint32_t sh = sbase + s_copy(0, 0), sl = sbase + s_copy(0, 1);
+      sts_bf2_split(sh + (gq * KP + col) * 2, sl + (gq * KP + col) * 2, st[j][0], st[j][1]);
+      sts_bf2_split(sh + ((gq + 8) * KP + col) * 2, sl + ((gq + 8) * KP + col) * 2, st[j][2], st[j][3]);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    for (int c = 0; c < n_chunks; ++c) {
+      const int sb = c & 1;
+      if (!tc::mbar_wait(full(c % L::NSTAGE), (uint32_t)((c / L::NSTAGE) & 1), abort_flag)) break;
+      const uint32_t base = sbase + stage_off(c);
+      const uint32_t kb = base + L::AW_B + L::Q_B;
+      const uint32_t upf = base + L::AW_B + L::Q_B + L::K_B + L::P_B;     // U' slice [C][DVS] fp32
+      const uint32_t gsa = upf + L::UPF_B;                                 // G [C] fp32
+      // 1a: Y = K S^T with S as hi + lo (m-tile mt, both n-tiles)
+      float cy[2][2][4] = {}, cyl[2][2][4] = {};               // [n-tile][k parity]
+      {
+        const uint32_t sh = sbase + s_copy(sb, 0) + b_s, sl = sbase + s_copy(sb, 1) + b_s;
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          uint32_t ak[4], bh[4], bl[4];
+          ldsm_x4_s(ak, kb + (ks >> 2) * L::HALF + a_off[ks & 3]);
+          ldsm_x4_s(bh, sh + ks * 32);
+          ldsm_x4_s(bl, sl + ks * 32);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            mma16816_h(cy[nt][ks & 1], ak, bh[2 * nt], bh[2 * nt + 1]);
+            mma16816_h(cyl[nt][ks & 1], ak, bl[2 * nt], bl[2 * nt + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[e] = (cy[nt][0][e] + cy[nt][1][e]) + (cyl[nt][0][e] + cyl[nt][1][e]);
+        const int col = nt * 8 + 2 * tq;
+        sts_bf2_split(sbase + yh + (r0 * UP + col) * 2, sbase + yl + (r0 * UP + col) * 2, y[0], y[1]);
+        sts_bf2_split(sbase + yh + (r1 * UP + col) * 2, sbase + yl + (r1 * UP + col) * 2, y[2], y[3]);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // the output warps are done with chunk c - 1: U buffer sb and state copy 1 - sb are free
+      if (c >= 1 && !tc::mbar_wait(done, (uint32_t)((c - 1) & 1), abort_flag)) break;
+      // 1b: W S^T = Aw Y with both as hi + lo (lo x lo dropped); U = U' - W S^T
+      const float Glast = lds_f(gsa + (C - 1) * 4);
+      const float e0 = expf(Glast - lds_f(gsa + r0 * 4)), e1 = expf(Glast - lds_f(gsa + r1 * 4)), gl = expf(Glast);
+      {
+        float cw[2][2][4] = {}, cx[2][2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+          uint32_t ah[4], al[4], bh[4], bl[4];
+          ldsm_x4_s(ah, base + a_off[ks]);
+          ldsm_x4_s(al, base + L::HALF + a_off[ks]);
+          ldsm_x4_t_s(bh, sbase + yh + b_y + ks * 16 * UP * 2);
+          ldsm_x4_t_s(bl, sbase + yl + b_y + ks * 16 * UP * 2);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            mma16816_h(cw[nt][ks & 1], ah, bh[2 * nt], bh[2 * nt + 1]);
+            mma16816_h(cx[nt][ks & 1], ah, bl[2 * nt], bl[2 * nt + 1]);
+            mma16816_h(cx[nt][ks & 1], al, bh[2 * nt], bh[2 * nt + 1]);
+          }
+        }
+        const uint32_t uo = sbase + u_out0 + sb * L::U_B;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int col = nt * 8 + 2 * tq;
+          float wv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) wv[e] = (cw[nt][0][e] + cw[nt][1][e]) + (cx[nt][0][e] + cx[nt][1][e]);
+          const float u00 = lds_f(upf + (r0 * DVS + col) * 4) - wv[0], u01 = lds_f(upf + (r0 * DVS + col + 1) * 4) - wv[1];
+          const float u10 = lds_f(upf + (r1 * DVS + col) * 4) - wv[2], u11 = lds_f(upf + (r1 * DVS + col + 1) * 4) - wv[3];
+          sts_bf2(uo + (r0 * UP + col) * 2, u00, u01);
+          sts_bf2(uo + (r1 * UP + col) * 2, u10, u11);
+          sts_bf2_split(sbase + ueh + (r0 * UP + col) * 2, sbase + uel + (r0 * UP + col) * 2, u00 * e0, u01 * e0);
+          sts_bf2_split(sbase + ueh + (r1 * UP + col) * 2, sbase + uel + (r1 * UP + col) * 2, u10 * e1, u11 * e1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(go(sb));                  // U of chunk c (and its start state) for the output warps
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // 3: S <- exp(G_last) S + (eU)^T K on this warp's dk columns
+      {
+        float s1[NT][4], l0[NT][4], l1[NT][4];
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            st[j][e] *= gl;
+            s1[j][e] = l0[j][e] = l1[j][e] = 0.f;
+          }
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+          uint32_t au[4], al[4];
+          ldsm_x4_t_s(au, sbase + ueh + a_ue + ks * 16 * UP * 2);
+          ldsm_x4_t_s(al, sbase + uel + a_ue + ks * 16 * UP * 2);
+#pragma unroll
+          for (int p = 0; p < NT / 2; ++p) {
+            uint32_t bk[4];
+            ldsm_x4_t_s(bk, kb + b_k[p] + ks * 16 * 128);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int j = 2 * p + q;
+              mma16816_h((ks & 1) ? s1[j] : st[j], au, bk[2 * q], bk[2 * q + 1]);
+              mma16816_h((ks & 1) ? l1[j] : l0[j], al, bk[2 * q], bk[2 * q + 1]);
+            }
+          }
+        }
+        const uint32_t sh = sbase + s_copy(sb ^ 1, 0), sl = sbase + s_copy(sb ^ 1, 1);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) st[j][e] += s1[j][e] + (l0[j][e] + l1[j][e]);
+          const int col = (cb + j) * 8 + 2 * tq;
+          sts_bf2_split(sh + (gq * KP + col) * 2, sl + (gq * KP + col) * 2, st[j][0], st[j][1]);
+          sts_bf2_split(sh + ((gq + 8) * KP + col) * 2, sl + ((gq + 8) * KP + col) * 2, st[j][2], st[j][3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(empty(c % L::NSTAGE));
+      asm volatile("bar.sync 1, 128;" ::: "memory");           // the new state copy, before the next Y
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int col = (cb + j) * 8 + 2 * tq;
+      Sg[gq * DK + col] = st[j][0];
+      Sg[gq * DK + col + 1] = st[j][1];
+      Sg[(gq + 8) * DK + col] = st[j][2];
+      Sg[(gq + 8) * DK + col + 1] = st[j][3];
+    }
+  } else {
+    // ---------------------------------------------------------------- output warps
+    for (int c = 0; c < n_chunks; ++c) {
+      const int sb = c & 1;
+      if (!tc::mbar_wait(full(c % L::NSTAGE), (uint32_t)((c / L::NSTAGE) & 1), abort_flag)) break;
+      if (!tc::mbar_wait(go(sb), (uint32_t)((c >> 1) & 1), abort_flag)) break;
+      const uint32_t base = sbase + stage_off(c);
+      const uint32_t qb = base + L::AW_B, pb = base + L::AW_B + L::Q_B + L::K_B;
+      const uint32_t gsa = base + L::AW_B + L::Q_B + L::K_B + L::P_B + L::UPF_B;
+      float cq[2][2][4] = {}, cp[2][2][4] = {};
+      const uint32_t sh = sbase + s_copy(sb, 0) + b_s;
+#pragma unroll
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        uint32_t aq[4], bs[4];
+        ldsm_x4_s(aq, qb + (ks >> 2) * L::HALF + a_off[ks & 3]);
+        ldsm_x4_s(bs, sh + ks * 32);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma16816_h(cq[nt][ks & 1], aq, bs[2 * nt], bs[2 * nt + 1]);
+      }
+      const uint32_t uo = sbase + u_out0 + sb * L::U_B + b_y;
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks) {
+        uint32_t ap[4], bu[4];
+        ldsm_x4_s(ap, pb + a_off[ks]);
+        ldsm_x4_t_s(bu, uo + ks * 16 * UP * 2);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma16816_h(cp[nt][ks & 1], ap, bu[2 * nt], bu[2 * nt + 1]);
+      }
+      const float g0 = expf(lds_f(gsa + r0 * 4)), g1 = expf(lds_f(gsa + r1 * 4));   // the last reads of the stage
+      const int c0 = c * C, n = min(C, T_len - c0);
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(done);                                 // U buffer sb and state copy sb may be reused
+        tc::mbar_arrive(empty(c % L::NSTAGE));
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int col = nt * 8 + 2 * tq;
+        if (r0 < n)
+          st_bf2(out + (((long)b * T_len + c0 + r0) * H + h) * DV + i0 + col,
+                 scale * fmaf(g0, cq[nt][0][0] + cq[nt][1][0], cp[nt][0][0] + cp[nt][1][0]),
+                 scale * fmaf(g0, cq[nt][0][1] + cq[nt][1][1], cp[nt][0][1] + cp[nt][1][1]));
+        if (r1 < n)
+          st_bf2(out + (((long)b * T_len + c0 + r1) * H + h) * DV + i0 + col,
+                 scale * fmaf(g1, cq[nt][0][2] + cq[nt][1][2], cp[nt][0][2] + cp[nt][1][2]),
+                 scale * fmaf(g1, cq[nt][0][3] + cq[nt][1][3], cp[nt][0][3] + cp[nt][1][3]));
+      }
+    }
   }
 }
 
@@ -1159,13 +1229,11 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
   constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;   // bf16: tensor-core sequential pass
   auto k1 = gdn_intra_kernel<T, DK, DV>;
   auto k2 = gdn_scan_kernel<T, DK, DV, DVS>;
-  auto k2t = gdn_scan_tc_kernel<DK, DV>;
   using L = ScanSmem<T, DK, DV, DVS>;
-  using LT = ScanTc<DK, DV>;
+  using LW = ScanWs<DK, DV>;
   {
     cudaError_t e = set_smem_limit(k1, (int)smem1);
     if (e == cudaSuccess) e = set_smem_limit(k2, (int)L::BYTES);
-    if (e == cudaSuccess) e = set_smem_limit(k2t, (int)LT::BYTES);
     if (e != cudaSuccess) return e;
   }
   if (TC) {
@@ -1196,7 +1264,7 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
     const cuuint64_t dG[2] = {GDN_C, nblk}, sG[1] = {bs};
     const cuuint64_t dQ[4] = {DK, (cuuint64_t)H, (cuuint64_t)T_len, (cuuint64_t)B};
     const cuuint64_t sQ[3] = {DK * 2, (cuuint64_t)H * DK * 2, (cuuint64_t)T_len * H * DK * 2};
-    const cuuint32_t b64[3] = {64, GDN_C, 1}, bA[3] = {64, 2 * GDN_C, 1}, bU[3] = {LT::DVS, GDN_C, 1},
+    const cuuint32_t b64[3] = {64, GDN_C, 1}, bA[3] = {64, 2 * GDN_C, 1}, bU[3] = {LW::DVS, GDN_C, 1},
                      bG[2] = {GDN_C, 1}, bQ[4] = {64, 1, GDN_C, 1};
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     if (!tc::make_map_nd(&mA, BF, 3, wsb + WLB::AW_OFF, dA, sA, bA, true) ||
@@ -1205,7 +1273,12 @@ static cudaError_t launch_two_pass(const void* q, const void* k, const void* v, 
         !tc::make_map_nd(&mG, F32, 2, wsb + WLB::G_OFF, dG, sG, bG, false) ||
         !tc::make_map_nd(&mQ, BF, 4, q, dQ, sQ, bQ, true) || !tc::make_map_nd(&mK, BF, 4, k, dQ, sQ, bQ, true))
       return cudaErrorNotSupported;
-    k2t<<<dim3(DV / LT::DVS, H, B), 256, LT::BYTES, s>>>(mA, mP, mU, mG, mQ, mK, state, (__nv_bfloat16*)out, T_len, H,
+    auto k2w = gdn_scan_ws_kernel<DK, DV>;
+    {
+      cudaError_t e2 = set_smem_limit(k2w, (int)LW::BYTES);
+      if (e2 != cudaSuccess) return e2;
+    }
+    k2w<<<dim3(DV / LW::DVS, H, B), 288, LW::BYTES, s>>>(mA, mP, mU, mG, mQ, mK, state, (__nv_bfloat16*)out, T_len, H,
                                                           n_chunks, scale);
   } else
     k2<<<dim3(DV / DVS, H, B), 256, L::BYTES, s>>>((const T*)q, (const T*)k, (const float*)workspace, state, (T*)out,

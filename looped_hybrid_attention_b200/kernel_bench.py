@@ -44,7 +44,8 @@ def main():
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
-    ap.add_argument("--epi", choices=["store", "add", "swiglu", "f32"], default="swiglu")
+    ap.add_argument("--epi", choices=["store", "add", "swiglu", "f32", "gdn"], default="swiglu",
+                    help="gdn: the GDN input projection with its preparation in the epilogue (N = 3*H*128 + 2*H)")
     ap.add_argument("--T", type=int, default=8192)
     ap.add_argument("--H", type=int, default=16)
     ap.add_argument("--B", type=int, default=1)
@@ -57,7 +58,19 @@ def main():
     bf = torch.bfloat16
     r = lambda *s, std=1.0: (std * torch.randn(*s, device=dev, generator=g)).to(bf)
     res = {"op": a.op}
-    if a.op == "gemm":
+    if a.op == "gemm" and a.epi == "gdn":
+        H = a.N // 386 if a.N % 386 == 0 else 16            # N = 3*H*128 + 2*H
+        N = 3 * H * 128 + 2 * H
+        X, W = r(a.M, a.K), r(N, a.K, std=0.02)
+        q = torch.empty((a.M, H, 128), device=dev, dtype=bf)
+        k, v = torch.empty_like(q), torch.empty_like(q)
+        gg, beta = torch.empty((a.M, H), device=dev), torch.empty((a.M, H), device=dev)
+        ab, bb = torch.zeros(H, device=dev), torch.zeros(H, device=dev)
+        ms = timed(lambda: L.gdn_in_proj(X, W, ab, bb, q, k, v, gg, beta, H, 128, 128, 1e-6), a.warmup, a.iters)
+        flops = 2.0 * a.M * N * a.K
+        byts = 2.0 * (a.M * a.K + N * a.K) + 2.0 * a.M * 3 * H * 128 + 8.0 * a.M * H
+        res.update(shape=[a.M, N, a.K], epi="gdn", ms=ms, tflops=flops / ms / 1e9, gbs=byts / ms / 1e6)
+    elif a.op == "gemm":
         X, W = r(a.M, a.K), r(a.N, a.K, std=0.02)
         W2 = r(a.N, a.K, std=0.02) if a.epi == "swiglu" else None
         R = r(a.M, a.N) if a.epi == "add" else None
