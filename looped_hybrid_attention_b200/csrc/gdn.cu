@@ -996,13 +996,14 @@ struct IntraTc {
   static constexpr int QA_B = (K_B > SPLIT_B ? K_B : SPLIT_B);      // Q, later the W factors
   static constexpr int AU_B = (C * FP * 4 > SPLIT_B ? C * FP * 4 : SPLIT_B);   // A, later the U' factors
   static constexpr int T_B = C * FP * 4, M_B = 3 * 256 * 4, G_B = 3 * C * 4;
-  static constexpr int OFF_K = 0, OFF_V = OFF_K + K_B, OFF_QA = OFF_V + V_B, OFF_AU = OFF_QA + QA_B,
-                       OFF_T = OFF_AU + AU_B, OFF_M = OFF_T + T_B, OFF_G = OFF_M + M_B;
-  static constexpr size_t BYTES = (size_t)OFF_G + G_B;
+  static constexpr int KT_B = K_B > T_B ? K_B : T_B;       // K, then T (K's last use is K K^T, Q K^T)
+  static constexpr int OFF_K = 0, OFF_T = 0, OFF_V = KT_B, OFF_QA = OFF_V + V_B, OFF_AU = OFF_QA + QA_B,
+                       OFF_M = OFF_AU + AU_B, OFF_G = OFF_M + M_B;
+  static constexpr size_t BYTES = (size_t)OFF_G + G_B;     // 75.5 KB at dk = dv = 128: three CTAs per SM
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, 3)
     gdn_intra_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                         const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                         const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int n_chunks) {
