@@ -274,9 +274,11 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
                                 EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
        "FA output projection");
   }
-  // u = x + mix; FFN on RMSNorm(u)
-  CK(prof(m, s, P_RMSNORM, 1, 0, es * (4.0 * M * d + d),
-          [&] { return rmsnorm(x, m->mix.p, m->u.p, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s); }),
+  // u = x + mix; FFN on RMSNorm(u).  Only plain layers add f to u (h = u + f); looped
+  // layers add it to mix (F = mix + f), so there u is not stored.
+  void* u_out = r.in_loop ? nullptr : m->u.p;
+  CK(prof(m, s, P_RMSNORM, 1, 0, es * ((u_out ? 4.0 : 3.0) * M * d + d),
+          [&] { return rmsnorm(x, m->mix.p, u_out, w.ffn_norm, m->un.p, (int)M, d, cf.eps, dt, s); }),
      "rmsnorm (FFN)");
   gemm_work(M, cf.ffn, d, EPI_SWIGLU, m->esize, fl, by);
   CK(prof(m, s, P_GEMM, 1, fl, by,

@@ -52,6 +52,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--no-ws", action="store_true", help="gemm: no partial-sum workspace (whole tiles per CTA)")
+    ap.add_argument("--rotate", type=int, default=1,
+                    help="gemm: cycle through this many weight copies (more than L2 holds: cold weights)")
+    ap.add_argument("--graph", action="store_true",
+                    help="gemm: time a CUDA graph of the launches (no host issue cost in the timing)")
     a = ap.parse_args()
     dev = torch.device("cuda")
     g = torch.Generator(device=dev).manual_seed(0)
@@ -71,15 +75,33 @@ def main():
         byts = 2.0 * (a.M * a.K + N * a.K) + 2.0 * a.M * 3 * H * 128 + 8.0 * a.M * H
         res.update(shape=[a.M, N, a.K], epi="gdn", ms=ms, tflops=flops / ms / 1e9, gbs=byts / ms / 1e6)
     elif a.op == "gemm":
-        X, W = r(a.M, a.K), r(a.N, a.K, std=0.02)
-        W2 = r(a.N, a.K, std=0.02) if a.epi == "swiglu" else None
+        X = r(a.M, a.K)
+        Ws = [r(a.N, a.K, std=0.02) for _ in range(a.rotate)]
+        W2s = [r(a.N, a.K, std=0.02) if a.epi == "swiglu" else None for _ in range(a.rotate)]
         R = r(a.M, a.N) if a.epi == "add" else None
         Y = torch.empty((a.M, a.N), device=dev, dtype=torch.float32 if a.epi == "f32" else bf)
         epi = {"store": L.EPI_STORE, "add": L.EPI_ADD, "swiglu": L.EPI_SWIGLU, "f32": L.EPI_F32}[a.epi]
         # zero-filled partial-sum workspace for few rows (M <= 128), as the runtime gives it
         nws = L.linear_workspace_bytes(a.M, a.N, a.K, epi)
         ws = torch.zeros(nws // 4 + 1, device=dev) if nws and not a.no_ws else None
-        ms = timed(lambda: L.linear(X, W, Y, epi, W2=W2, R=R, workspace=ws), a.warmup, a.iters)
+        it = [0]
+
+        def call():
+            i = it[0] % a.rotate
+            it[0] += 1
+            L.linear(X, Ws[i], Y, epi, W2=W2s[i], R=R, workspace=ws)
+
+        if a.graph:
+            for _ in range(a.warmup):
+                call()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(a.iters):
+                    call()
+            ms = timed(graph.replay, 2, 1) / a.iters
+        else:
+            ms = timed(call, a.warmup, a.iters)
         nmat = 2 if a.epi == "swiglu" else 1
         flops = 2.0 * a.M * a.N * a.K * nmat
         byts = 2.0 * (a.M * a.K + nmat * a.N * a.K) + Y.element_size() * a.M * a.N * (2 if a.epi == "add" else 1)
