@@ -552,7 +552,8 @@ def run_ours(args, world, rank, local):
                          "roofline_kernel": leg["roofline"]["kernel"], "roofline_frac": leg["roofline"]["frac"],
                          "sm_mhz": leg["clocks"]["sm_mhz"]}
             if "step_roofline" in leg:
-                legs[key]["step_frac_of_hbm_roofline"] = leg["step_roofline"]["frac"]
+                sr = leg["step_roofline"]
+                legs[key][f"step_frac_of_{sr['bound']}_roofline"] = sr["frac"]
     line["legs"] = legs
     print(json.dumps(line), flush=True)
 

@@ -65,7 +65,18 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
   // VEC: rows 16-byte aligned, so each lane moves its PER elements as 8-element vectors
   constexpr bool V8 = VEC && PER % 8 == 0;
   float x[R][PER], gn[PER];
+  // key rows: their values' 16-byte pieces are loaded together with the keys (one round trip)
+  constexpr int VP = V8 ? PER * (int)sizeof(T) / 16 : 1;
+  uint4 vv[R][VP];
+  const T* vsrc = row + 2 * Hq * DH + Hkv * DH + kvh0 * DH;
   if constexpr (V8) {
+    if (!is_q) {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int i = 0; i < VP; ++i)
+          vv[r][i] = *reinterpret_cast<const uint4*>(vsrc + r * DH + lane * PER + i * (16 / (int)sizeof(T)));
+    }
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -134,12 +145,12 @@ __global__ void __launch_bounds__(256) fa_prep_kernel(const T* __restrict__ P, i
     } else {
       const long slot = (((long)b * Hkv + kvh0 + r) * kv_cap + pos) * DH;
       dst = k_cache + slot;
-      const T* vs = row + 2 * Hq * DH + Hkv * DH + (kvh0 + r) * DH;
+      const T* vs = vsrc + r * DH;
       T* vd = v_cache + slot;
       if constexpr (V8) {
 #pragma unroll
-        for (int u = 0; u < PER; u += 16 / (int)sizeof(T))
-          *reinterpret_cast<uint4*>(vd + lane * PER + u) = *reinterpret_cast<const uint4*>(vs + lane * PER + u);
+        for (int i = 0; i < VP; ++i)
+          *reinterpret_cast<uint4*>(vd + lane * PER + i * (16 / (int)sizeof(T))) = vv[r][i];
       } else {
 #pragma unroll
         for (int u = 0; u < PER; ++u) vd[lane * PER + u] = vs[lane * PER + u];
