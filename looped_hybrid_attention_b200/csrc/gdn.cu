@@ -1411,6 +1411,111 @@ __global__ void __launch_bounds__(256) gdn_step_kernel(const T* __restrict__ q, 
   }
 }
 
+// The decode step straight from the stored input projection (rows q | k | v | a | b per
+// token, H heads): each warp L2-normalises its head's q and k (eps inside the root) and
+// rounds them to the storage type, forms g = -softplus(a + a_bias) and beta = sigmoid(b +
+// b_bias) -- what the GDN preparation would have stored -- then updates its R state rows as
+// gdn_step_kernel does.  The preparation's launch and its q, k, v, g, beta round trip are
+// gone from the decode step.
+template <typename T, int DK, int R, bool VEC>
+__global__ void __launch_bounds__(256) gdn_step_proj_kernel(const T* __restrict__ P, int ld_p,
+                                                            const float* __restrict__ a_bias,
+                                                            const float* __restrict__ b_bias, float eps, int H,
+                                                            float* __restrict__ state, T* __restrict__ out, int BH,
+                                                            int DV, float scale) {
+  pdl_trigger();
+  constexpr int PER = DK / 32;
+  const int lane = threadIdx.x & 31;
+  const long row0 = ((long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * R;
+  if (row0 >= (long)BH * DV) return;
+  const long bh = row0 / DV;                     // DV % R == 0: the R rows share the head
+  const int i0 = (int)(row0 % DV);
+  const long b = bh / H;
+  const int h = (int)(bh % H);
+  const T* prow = P + b * ld_p;
+  float* S = state + row0 * DK + lane * PER;
+  float s[R][PER], kk[PER], qq[PER];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (VEC) {
+      Vec<PER>::ld(S + r * DK, s[r]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < PER; ++u) s[r][u] = S[r * DK + u];
+    }
+  }
+  float sq = 0.f, sk = 0.f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    qq[u] = ldf(prow + (long)h * DK + lane * PER + u);
+    kk[u] = ldf(prow + (long)(H + h) * DK + lane * PER + u);
+    sq = fmaf(qq[u], qq[u], sq);
+    sk = fmaf(kk[u], kk[u], sk);
+  }
+  const T* gates = prow + 2L * H * DK + (long)H * DV;
+  const float a = ldf(gates + h) + a_bias[h];
+  const float bb = ldf(gates + H + h) + b_bias[h];
+  const float iq = rsqrtf(warp_sum(sq) + eps), ik = rsqrtf(warp_sum(sk) + eps);
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    qq[u] = Io<T>::round(qq[u] * iq);
+    kk[u] = Io<T>::round(kk[u] * ik);
+  }
+  const float sp = a > 20.f ? a : log1pf(expf(a));    // softplus
+  const float alpha = expf(-sp), bt = 1.f / (1.f + expf(-bb));
+  const T* vrow = prow + 2L * H * DK + (long)h * DV;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float pred = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) pred = fmaf(s[r][u], kk[u], pred);
+    pred = warp_sum(pred) * alpha;
+    const float uu = bt * (ldf(vrow + i0 + r) - pred);
+    float o = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      s[r][u] = fmaf(alpha, s[r][u], uu * kk[u]);
+      o = fmaf(s[r][u], qq[u], o);
+    }
+    if (VEC) {
+      Vec<PER>::st(S + r * DK, s[r]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < PER; ++u) S[r * DK + u] = s[r][u];
+    }
+    o = warp_sum(o);
+    if (lane == 0) stf(out + bh * DV + i0 + r, scale * o);
+  }
+}
+
+cudaError_t gdn_step_proj(const void* P, int ld_p, const float* a_bias, const float* b_bias, float eps, float* state,
+                          void* out, int B, int H, int dk, int dv, float scale, int dtype, cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
+  const long rows = (long)B * H * dv;
+  const bool r4 = dv % 4 == 0 && (uintptr_t)state % (dk == 128 ? 16 : 8) == 0;
+  const dim3 grid((unsigned)((rows + (r4 ? 31 : 7)) / (r4 ? 32 : 8)));
+#define GDN_STEP_P(TT, DKK, RR)                                                                             \
+  gdn_step_proj_kernel<TT, DKK, RR, (RR > 1)><<<grid, 256, 0, s>>>((const TT*)P, ld_p, a_bias, b_bias, eps, H, \
+                                                                   state, (TT*)out, B * H, dv, scale)
+  if (dk == 128) {
+    if (dtype == BF16) {
+      if (r4) GDN_STEP_P(__nv_bfloat16, 128, 4); else GDN_STEP_P(__nv_bfloat16, 128, 1);
+    } else {
+      if (r4) GDN_STEP_P(float, 128, 4); else GDN_STEP_P(float, 128, 1);
+    }
+  } else if (dk == 64) {
+    if (dtype == BF16) {
+      if (r4) GDN_STEP_P(__nv_bfloat16, 64, 4); else GDN_STEP_P(__nv_bfloat16, 64, 1);
+    } else {
+      if (r4) GDN_STEP_P(float, 64, 4); else GDN_STEP_P(float, 64, 1);
+    }
+  } else {
+    return cudaErrorNotSupported;
+  }
+#undef GDN_STEP_P
+  return cudaGetLastError();
+}
+
 cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      float* state, void* out, int B, int H, int dk, int dv, float scale, int dtype,
                      cudaStream_t s) {

@@ -65,6 +65,10 @@ size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t gdn_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                      float* state, void* out, int B, int H, int dk, int dv, float scale, int dtype,
                      cudaStream_t s);
+// Decode step from the stored input projection (q | k | v | a | b rows): the GDN preparation
+// (L2 norms, gates) happens inside the step.
+cudaError_t gdn_step_proj(const void* P, int ld_p, const float* a_bias, const float* b_bias, float eps, float* state,
+                          void* out, int B, int H, int dk, int dv, float scale, int dtype, cudaStream_t s);
 bool gdn_supported(int dk, int dv);
 // GDN variant (short causal conv + gated output norm; Hv value heads reading Hk key heads)
 bool gdn_variant_supported(int Hk, int Hv, int dk, int dv, int conv);

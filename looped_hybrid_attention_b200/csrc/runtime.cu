@@ -192,7 +192,9 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
                                   d, EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
          "GDN input projection");
     }
-    if (fused_prep) {
+    // the decode step reads the stored projection itself (norms and gates inside the step)
+    const bool step_from_proj = !fused_prep && !variant && T == 1;
+    if (fused_prep || step_from_proj) {
     } else if (variant) {
       void* conv_state = (char*)c->conv.p + (size_t)r.slot * c->conv_elems * m->esize;
       // P's q | k | v channels read conv times, the conv inputs before this call, outputs once
@@ -214,7 +216,13 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
     // bytes: q, k, v in, o out, gates, and the fp32 state read + written once
     const double st_bytes = 8.0 * B * H * dk * dv;
     const double io_bytes = (double)M * H * (es * (2.0 * dk + 2.0 * dv) + 8.0);
-    if (T == 1)
+    if (step_from_proj)
+      CK(prof(m, s, P_GDN_STEP, 1, 6.0 * B * H * dk * dv,
+              (double)M * (es * (2.0 * H * dk + H * dv + 2.0 * H + H * dv)) + st_bytes,
+              [&] { return lk::gdn_step_proj(m->proj.p, m->in_gdn, w.gdn_a_bias, w.gdn_b_bias, cf.eps, S, m->o.p, B, H,
+                                             dk, dv, scale, dt, s); }),
+         "GDN step");
+    else if (T == 1)
       CK(prof(m, s, P_GDN_STEP, 1, 6.0 * B * H * dk * dv, io_bytes + st_bytes,
               [&] { return lk::gdn_step(m->gq.p, m->gk.p, m->gv.p, (float*)m->gg.p, (float*)m->gb.p, S, m->o.p, B, H,
                                         dk, dv, scale, dt, s); }),

@@ -154,7 +154,11 @@ def main():
         x, rr, w = r(M, d), r(M, d), r(d)
         y, sm = torch.empty_like(x), torch.empty_like(x)
         ms = timed(lambda: L.rmsnorm(x, w, y, 1e-6, r=rr, sum_out=sm), a.warmup, a.iters)
-        res.update(shape=[M, d], ms=ms, gbs=2.0 * 4 * M * d / ms / 1e6)
+        ms_add = timed(lambda: L.rmsnorm(x, w, y, 1e-6, r=rr), a.warmup, a.iters)
+        ms_plain = timed(lambda: L.rmsnorm(x, w, y, 1e-6), a.warmup, a.iters)
+        res.update(shape=[M, d], ms=ms, gbs=2.0 * 4 * M * d / ms / 1e6,
+                   add_no_sum_ms=ms_add, add_no_sum_gbs=2.0 * 3 * M * d / ms_add / 1e6,
+                   plain_ms=ms_plain, plain_gbs=2.0 * 2 * M * d / ms_plain / 1e6)
     elif a.op == "gdnprep":
         M, H, dk = a.M, a.H, 128
         n_in = 3 * H * dk + 2 * H
