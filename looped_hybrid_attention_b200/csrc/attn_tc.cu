@@ -358,25 +358,27 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       // the row maximum of the tile (every processed tile but a last partial one has a
       // visible key per row; a row without one gets P = 0 there)
       const float mt = fmaxf(mh, xmax[(s * 2 + (half ^ 1)) * AT_M + r]) * scale_log2;
-      if (mt > m_used + RESCALE_THRESHOLD) {
-        if (j > 0) {                                  // O holds tiles < j scaled by 2^-m_used
-          if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) goto done;
-          const float corr = exp2f(m_used - mt);
-          l *= corr;
-          fence_after();
+      const bool grow = mt > m_used + RESCALE_THRESHOLD;
+      // O holds tiles < j scaled by 2^-m_used.  The TMEM loads and stores are warp-wide
+      // instructions, so the whole warp rescales when any of its rows must (the others
+      // with factor 1, which leaves O unchanged); the two threads of a row decide alike.
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (!mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) goto done;
+        const float corr = grow ? exp2f(m_used - mt) : 1.f;
+        l *= corr;
+        fence_after();
 #pragma unroll 1
-          for (int c = 0; c < AT_D / 64; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + lane_off + half * (AT_D / 2) + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < AT_D / 64; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + half * (AT_D / 2) + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-            tmem_st32(tO + lane_off + half * (AT_D / 2) + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st32(tO + lane_off + half * (AT_D / 2) + c * 32, o);
         }
-        m_used = mt;
+        tmem_wait_st();
       }
+      if (grow) m_used = mt;
       // this half's 64 keys of P as bf16 pairs (key 2i in the low half of column i) into
       // columns [32 half, 32 half + 32) of this tile's S buffer, the A operand of P V
       // (packed f32x2 FMAs and adds: two scores per instruction)

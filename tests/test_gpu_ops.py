@@ -607,6 +607,35 @@ def test_attention_single_key_and_zero_query(cuda):
     assert torch.allclose(out.view(T, Hq, dh)[0], Vc[0, 0, 0][None].expand(Hq, dh), atol=1e-6)
 
 
+def test_attention_late_dominant_key_rescales_part_of_a_warp(cuda):
+    """One key in the third 128-key tile is scaled up 12x, so the running row maximum of about
+    a quarter of the query rows jumps by far more than the lazy-rescale threshold there while
+    the other rows of the same warps keep theirs: O is rescaled for some rows of a warp only.
+    Every row against brute force."""
+    import looped_hybrid_attention_b200 as L
+    T, Hq, Hkv, dh = 600, 16, 4, 256
+    q = rnd((T, Hq, dh), 53, "qd", dtype="bf16")
+    Kc = rnd((1, Hkv, T, dh), 54, "Kd")
+    Kc[0, :, 300] *= 12.0
+    Kc = Kc.to(torch.bfloat16)
+    Vc = rnd((1, Hkv, T, dh), 55, "Vd", dtype="bf16")
+    out = torch.empty((T, Hq * dh), dtype=torch.bfloat16, device=cuda)
+    L.gqa_attn(q, Hq * dh, Kc, Vc, T, None, 0, out, 1, T, T, 0, Hq, Hkv, dh, True)
+    torch.cuda.synchronize()
+    # rows t >= 300 whose score at key 300 exceeds their maximum over keys 0..255 (the first
+    # two tiles) by more than 8 in log2 units: those rescale O at the third tile
+    qn, Kn = to64(q), to64(Kc[0])
+    kv = np.arange(Hq) // (Hq // Hkv)
+    s_late = np.einsum("thd,hd->th", qn[300:], Kn[kv, 300]) / 16.0
+    s_early = np.einsum("thd,hkd->thk", qn[300:], Kn[kv, :256]) / 16.0
+    jump = (s_late - s_early.max(axis=-1)) * np.log2(np.e)
+    frac = float(np.mean(jump > 8.0))
+    assert 0.05 < frac < 0.95, frac                  # some rows of a warp rescale, others do not
+    ref = ops.attention(to64(q), to64(Kc[0]).transpose(1, 0, 2), to64(Vc[0]).transpose(1, 0, 2), np.arange(T))
+    assert rel_l2(to64(out).reshape(T, Hq, dh), ref) < TOL["bf16"]
+    assert L.device_error() == 0
+
+
 @pytest.mark.slow
 def test_attention_full_length_sampled_rows(cuda):
     """The bench's shape (T = 8192, 16q/4kv x 256, bf16): sampled query rows against brute force."""
