@@ -359,6 +359,40 @@ def test_gdn_step_layouts(cuda, dtype, dk, dv, offset):
         assert rel_l2(to64(S[b]), S_ref) < STATE_TOL[dtype]
 
 
+@pytest.mark.parametrize("two_pass", [False, True])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_gdn_extreme_gates(cuda, dtype, two_pass):
+    """Gates far from the random-init range: decays from ~1 down to exp(-75) per token (a
+    chunk's cumulative log decay reaches the thousands, so many exp(G) underflow to 0), and
+    write strengths beta pressed against 0 and 1.  The chunked form never divides by a decay,
+    so it must stay finite and match the recurrence."""
+    import looped_hybrid_attention_b200 as L
+    B, T, H, dk = 1, 300, 2, 128
+    q, k, v, _, _, S = _gdn_inputs(B, T, H, dk, dk, dtype, seed=77)
+    a = synth.normal((B, T, H), 25.0, 77, "a_x").double().numpy()
+    bb = synth.normal((B, T, H), 10.0, 77, "b_x").double().numpy()
+    g_np, beta_np = ops.gdn_gates(a, bb, 0.0, 0.0)
+    g = torch.tensor(g_np, dtype=torch.float32, device=cuda)
+    beta = torch.tensor(beta_np, dtype=torch.float32, device=cuda)
+    assert g_np.min() < -50 and (beta_np < 1e-3).any() and (beta_np > 1 - 1e-3).any()
+    S0 = S.clone()
+    out = torch.empty_like(v)
+    scale = 1.0 / np.sqrt(dk)
+    ws = torch.empty(L.gdn_workspace_bytes(B, T, H, dk, dk) // 4, device=cuda) if two_pass else None
+    L.gdn_chunk_fwd(q, k, v, g, beta, S, out, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(S).all()
+    o_ref, S_ref = ops.gdn_recurrent(to64(q[0]), to64(k[0]), to64(v[0]), to64(g[0]), to64(beta[0]), to64(S0[0]),
+                                     scale)
+    # fp32: the chunked form takes each decay exp(G_r - G_s) from the chunk's fp32 cumulative
+    # log decays G, so an exponent carries an absolute error up to about |G| 2^-24 -- here
+    # |G| reaches 64 * 76 ~ 4,900, i.e. ~3e-4 -- which the recurrence (one factor per token)
+    # does not have; the bound for these gates is 1e-4 instead of the 1e-5 of the ordinary range
+    tol = 1e-4 if dtype == "fp32" else TOL[dtype]
+    assert rel_l2(to64(out[0]), o_ref) < tol
+    assert rel_l2(to64(S[0]), S_ref) < 1e-4            # the fp32-grade state bound of both paths
+
+
 def test_gdn_special_cases(cuda):
     import looped_hybrid_attention_b200 as L
     B, T, H, dk = 1, 100, 2, 64
