@@ -302,7 +302,8 @@ loop_status gqa_attn_noalloc(const void* q, int ld_q, const void* k, const void*
  * are the slab as fa_prep writes it (keys already normed and rotated).  Built for the
  * tensor-core kernel only: bf16, dh 256, Tq >= 16, 128 % (Hq/Hkv) == 0, rotary_dims <=
  * dh/2, 16-byte aligned q, q_norm, k, v, gate; other calls return LOOP_ERR_UNSUPPORTED.
- * Needs no workspace. */
+ * Needs no workspace.  The rotary angles are evaluated in fp64 by each query row's
+ * threads (the model's own forward passes a per-call cos/sin table instead). */
 loop_status gqa_attn_fused_q(const void* q, int ld_q, const void* q_norm, int rotary_dims, float rope_base,
                              float eps, const void* k, const void* v, int kv_cap, const void* gate,
                              int ld_gate, void* out, int B, int Tq, int Tkv, int q_off, int Hq, int Hkv,
