@@ -41,7 +41,12 @@ constexpr int Q_BYTES = AT_M * AT_D * 2;            // 64 KiB: four [128 rows][6
 constexpr int SLOT = 16384;                         // K quarter [128 keys][64 dims] or V [4][32 keys][64 dims]
 constexpr int N_SLOTS = 9;
 constexpr int XCH_BYTES = 2 * AT_M * 4 + 4 * AT_M * 4;   // row sums [2][128]; half-row maxima [2][2][128]
-constexpr int AT_SMEM = Q_BYTES + N_SLOTS * SLOT + 1024 + 256 + XCH_BYTES;
+// query staging with QK-norm and rotary: the norm gain [256] bf16, and the cos/sin rows of
+// the CTA's query positions ([QT <= 32][RT_MAX + 1] float2: one pad entry per row keeps the
+// rows' same entries in different banks) when rot <= 2 * RT_MAX
+constexpr int RT_MAX = 32, STAB_ROWS = 32;
+constexpr int GAIN_BYTES = AT_D * 2, STAB_BYTES = STAB_ROWS * (RT_MAX + 1) * 8;
+constexpr int AT_SMEM = Q_BYTES + N_SLOTS * SLOT + 1024 + 256 + XCH_BYTES + GAIN_BYTES + STAB_BYTES;
 constexpr int AT_THREADS = 320;                  // TMA, MMA, two softmax warpgroups
 // mbarrier slots
 constexpr int B_Q = 0, B_F = 1, B_E = B_F + N_SLOTS, B_SF = B_E + N_SLOTS, B_PF = B_SF + 2, B_PV = B_PF + 2,
@@ -57,6 +62,17 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 8 bf16 (one 16-byte piece) -> 8 floats.
+__device__ __forceinline__ void unpack8_bf16(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
 }
 
 // Two fp32 FMAs / adds as one packed instruction (each lane rounds exactly as fmaf / +).
@@ -90,6 +106,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint32_t* tmem_slot = (uint32_t*)(bars + N_BARS);
   float* xsum = (float*)((uint8_t*)bars + 256);        // row-sum exchange [2 halves][AT_M]
   float* xmax = xsum + 2 * AT_M;                       // half-row maxima [tile parity][half][AT_M]
+  uint4* sgain = reinterpret_cast<uint4*>(xmax + 4 * AT_M);   // query norm gain (fused query staging)
+  float2* stab = reinterpret_cast<float2*>(sgain + AT_D / 8);  // cos/sin rows of the CTA's positions
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0 + 8u * B_Q;
@@ -259,8 +277,78 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           const int dim = 128 * half + 8 * c;
           put(dim, ok ? src[dim >> 3] : make_uint4(0, 0, 0, 0));
         }
+      } else if (rot / 2 <= RT_MAX && QT <= STAB_ROWS) {
+        // Every global load of the staging in one round trip: this thread's raw half-row
+        // (kept in registers), and, shared by the CTA, the norm gain and the cos/sin rows of
+        // its QT positions (from the forward's table, coalesced, or evaluated here in fp64)
+        // into shared memory.  Then the row's sum of squares is exchanged with the other
+        // half's thread, and the rows are normalised and rotated from registers and shared
+        // memory.
+        const int tid_s = threadIdx.x - 64;             // 0..255
+        const int rt = rot / 2;
+        uint4 raw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) raw[c] = ok ? src[16 * half + c] : make_uint4(0, 0, 0, 0);
+        if (tid_s < AT_D / 8) sgain[tid_s] = reinterpret_cast<const uint4*>(q_norm)[tid_s];
+        for (int i = tid_s; i < QT * rt; i += 256) {
+          const int qr = i / rt, jp = i - qr * rt;
+          float2 t2 = make_float2(1.f, 0.f);
+          if (q0 + qr < Tq) {
+            const int p = q_off + q0 + qr;
+            if (rope_tab) {
+              t2 = rope_tab[(long)(p - tab_pos0) * rt + jp];
+            } else {
+              const double theta = pow((double)rope_base, -2.0 * (double)jp / (double)rot);
+              double ang = (double)p * theta;
+              ang -= 6.283185307179586 * floor(ang / 6.283185307179586);
+              double sd, cd;
+              sincos(ang, &sd, &cd);
+              t2 = make_float2((float)cd, (float)sd);
+            }
+          }
+          stab[qr * (RT_MAX + 1) + jp] = t2;
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float x8[8];
+          unpack8_bf16(raw[c], x8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(x8[e], x8[e], ss);
+        }
+        xsum[half * AT_M + r] = ss;
+        asm volatile("bar.sync 1, 256;" ::: "memory");     // the 256 softmax threads: sums, gain, table
+        const float inv = rsqrtf((xsum[r] + xsum[AT_M + r]) * (1.f / AT_D) + eps);
+        asm volatile("bar.sync 1, 256;" ::: "memory");     // both read before xsum is reused
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int dim = 128 * half + 8 * c;
+          float x8[8], g8[8];
+          unpack8_bf16(raw[c], x8);
+          unpack8_bf16(sgain[dim >> 3], g8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x8[e] = x8[e] * inv * g8[e];
+          if (dim < rot) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const float2 t2 = stab[qi * (RT_MAX + 1) + ((dim + e) >> 1)];
+              const float a0 = x8[e], a1 = x8[e + 1];
+              x8[e] = a0 * t2.x - a1 * t2.y;
+              x8[e + 1] = a0 * t2.y + a1 * t2.x;
+            }
+          }
+          uint4 v4;
+          uint32_t* pw = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(x8[2 * e], x8[2 * e + 1]);
+            pw[e] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          put(dim, v4);
+        }
       } else {
-        // raw row: this half's sum of squares, exchanged with the other half's thread
+        // other head groupings or rotary widths: two passes over the raw row (sum of
+        // squares, then scale and rotate), the angles from the table or in fp64
         float ss = 0.f;
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
