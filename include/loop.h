@@ -118,6 +118,15 @@ typedef struct loop_cache loop_cache;
 const char* loop_last_error(void);
 /* Device error word (see Conventions); reads and clears it on the current device. */
 loop_status loop_device_error(int* code_out /* host */);
+
+/* Self-test of the bounded-wait error path: launches one CTA on `stream` in which a thread
+ * waits on an mbarrier that nothing completes.  After `cycles` SM clock cycles (0 < cycles
+ * <= 4e9; every wait inside the library's kernels gives up after 4e9, about 2 s) the wait
+ * gives up, records the wait-timeout code in the device error word and the kernel returns
+ * normally: the next loop_device_error() reports LOOP_ERR_TIMEOUT and clears it, and the
+ * context stays usable.  Nothing else is touched.  Returns LOOP_ERR_INVALID_ARG for cycles
+ * out of range, else the launch status. */
+loop_status loop_wait_selftest(long long cycles, void* stream);
 const char* loop_version(void);
 
 /* ---------------------------------------------------------------- schedule

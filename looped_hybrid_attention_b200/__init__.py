@@ -64,6 +64,7 @@ _SIGS = {
     "loop_last_error": ([], ctypes.c_char_p),
     "loop_version": ([], ctypes.c_char_p),
     "loop_device_error": ([ctypes.POINTER(ctypes.c_int)], _I),
+    "loop_wait_selftest": ([ctypes.c_longlong, _P], _I),
     "loop_schedule": ([ctypes.POINTER(loop_config), _P, _I, _P, _P, _P], _I),
     "loop_model_create": ([ctypes.POINTER(loop_config), ctypes.POINTER(loop_weights), ctypes.POINTER(_P)], _I),
     "loop_model_destroy": ([_P], _I),
@@ -160,6 +161,17 @@ def device_error() -> int:
     c = ctypes.c_int(0)
     _lib.loop_device_error(ctypes.byref(c))
     return c.value
+
+
+def device_error_status() -> int:
+    """loop_device_error's status (LOOP_ERR_TIMEOUT after a bounded wait gave up); clears the code."""
+    c = ctypes.c_int(0)
+    return _lib.loop_device_error(ctypes.byref(c))
+
+
+def wait_selftest(cycles, stream=None):
+    """One bounded wait that runs out after `cycles` SM clock cycles (the error path's self-test)."""
+    check(_lib.loop_wait_selftest(int(cycles), _stream(stream)), "loop_wait_selftest")
 
 
 def make_config(shape) -> loop_config:

@@ -2,6 +2,7 @@
 // All three are HBM-bound: one pass over their inputs with 16-byte accesses.
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace lk {
 
@@ -89,6 +90,28 @@ __global__ void __launch_bounds__(256) rmsnorm_reg_kernel(const T* __restrict__ 
     for (int i = 0; i < 8; ++i) o[i] = a[c][i] * inv * g[i];
     store8(y + base + j, o);
   }
+}
+
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that nothing
+// completes.  After `limit` clock cycles the wait gives up, records DEV_WAIT_TIMEOUT in the
+// device error word and the kernel returns normally, as every bounded wait in the library
+// does -- the host reads the code with loop_device_error and the context stays usable.
+__global__ void wait_selftest_kernel(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = tc::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(b, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) tc::mbar_wait(b, 0, &abort_flag, limit);   // phase 0 never completes
+}
+
+cudaError_t wait_selftest(long long limit, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(limit);
+  return cudaGetLastError();
 }
 
 cudaError_t rmsnorm(const void* x, const void* r, void* sum_out, const void* w, void* y, int M,

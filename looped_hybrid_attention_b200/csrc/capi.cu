@@ -51,6 +51,11 @@ loop_status loop_device_error(int* code_out) {
   return *code_out == DEV_WAIT_TIMEOUT ? LOOP_ERR_TIMEOUT : LOOP_OK;
 }
 
+loop_status loop_wait_selftest(long long cycles, void* stream) {
+  REQUIRE(cycles > 0 && cycles <= 4000000000LL, LOOP_ERR_INVALID_ARG, "cycles must be in (0, 4e9]");
+  return launched(lk::wait_selftest(cycles, S(stream)), "loop_wait_selftest");
+}
+
 static loop_status check_config(const loop_config* c) {
   REQUIRE(c, LOOP_ERR_INVALID_ARG, "config is NULL");
   REQUIRE(dtype_ok(c->dtype), LOOP_ERR_INVALID_ARG, "dtype must be LOOP_F32 or LOOP_BF16");

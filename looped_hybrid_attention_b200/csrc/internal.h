@@ -127,5 +127,7 @@ cudaError_t transpose_wr(const float* w, float* wt, int two_d, cudaStream_t s);
 cudaError_t sinkhorn(const float* logits, float* out, int N, int n, int iters, cudaStream_t s);
 
 int read_and_clear_device_error();
+// One bounded wait that runs out after `limit` SM clock cycles (the error path's self-test).
+cudaError_t wait_selftest(long long limit, cudaStream_t s);
 
 }  // namespace lk

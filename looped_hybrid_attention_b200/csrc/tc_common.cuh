@@ -34,14 +34,16 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the other side gave up (abort flag) or the wait ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait: false if the other side gave up (abort flag) or the wait ran out (after
+// `limit` SM clock cycles; it then records DEV_WAIT_TIMEOUT and sets the abort flag).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = WAIT_CYCLES) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > WAIT_CYCLES) {
+    if (clock64() - t0 > limit) {
       set_device_error(DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
       return false;

@@ -110,6 +110,9 @@ def test_newer_entry_points_argument_errors_without_gpu():
     assert L._lib.gdn_in_proj(*proj(8192, 4096, 16, 0)) == 7
     assert L._lib.gdn_in_proj(*proj(8192, 4096, 15, 1)) == 7
     assert L._lib.gdn_in_proj(*proj(8192, 4000, 16, 1)) == 2
+    # the bounded-wait self-test refuses a cycle limit outside (0, 4e9] before launching
+    assert L._lib.loop_wait_selftest(0, None) == 1
+    assert L._lib.loop_wait_selftest(5_000_000_000, None) == 1
     # gqa_attn_fused_q: the query norm gain is required; rotary dims even and at most dh / 2
     fq = lambda qn, rot: (P, 4096, qn, rot, 1e4, 1e-6, P, P, 64, P, 4096, P, 1, 64, 64, 0, 16, 4, 256, 1, 1, None)
     assert L._lib.gqa_attn_fused_q(*fq(None, 64)) == 1
