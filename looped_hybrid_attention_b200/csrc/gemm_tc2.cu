@@ -133,11 +133,80 @@ __device__ __forceinline__ void gdn_epilogue(uint32_t t_row, int row, int n0, in
   }
 }
 
+// EPI_FA: one row's 256 columns (one head or a 256-column piece of the gate / v block) from
+// TMEM (8 loads of 32).  q and k heads: sum of squares, then scaled by rsqrt(mean + eps)
+// and the gain, the first `rot` dims rotated in adjacent pairs, stored (k into the slab);
+// gate and v pieces copied.  The TMEM loads are warp-collective: every lane issues them,
+// and only the stores are guarded by the row.
+__device__ __forceinline__ void fa_epilogue(uint32_t t_row, int row, int n0, int M, const FaEpi& fe) {
+  constexpr int D = 256;
+  const bool ok = row < M;
+  const int qe = fe.Hq * D, ge = 2 * qe, ke = ge + fe.Hkv * D;
+  const int b = ok ? row / fe.T : 0, t = ok ? row % fe.T : 0;
+  const long pos = (long)fe.pos0 + t;
+  const bool norm = n0 < qe || (n0 >= ge && n0 < ke);
+  __nv_bfloat16* dst;
+  if (n0 < qe) dst = (__nv_bfloat16*)fe.q + ((long)row * fe.Hq + n0 / D) * D;
+  else if (n0 < ge) dst = (__nv_bfloat16*)fe.gate + (long)row * fe.ld_gate + (n0 - qe);
+  else if (n0 < ke) dst = (__nv_bfloat16*)fe.k_slab + (((long)b * fe.Hkv + (n0 - ge) / D) * fe.kv_cap + pos) * D;
+  else dst = (__nv_bfloat16*)fe.v_slab + (((long)b * fe.Hkv + (n0 - ke) / D) * fe.kv_cap + pos) * D;
+  float inv = 1.f;
+  if (norm) {
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(t_row + c * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
+    }
+    inv = rsqrtf(ss * (1.f / D) + fe.eps);
+  }
+  const __nv_bfloat16* gain = (const __nv_bfloat16*)(n0 < qe ? fe.q_gain : fe.k_gain);
+  const int rh = fe.rot / 2;
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_row + c * 32, r);
+    tmem_wait_ld();
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    if (norm) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        float g8[8];
+        load8(gain + c * 32 + i, g8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[i + e] = v[i + e] * inv * g8[e];
+      }
+      if (c * 32 < fe.rot) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int j = (c * 32 + i) >> 1;
+          if (j < rh) {
+            const float2 cs = fe.rope[(long)t * rh + j];
+            const float a0 = v[i], a1 = v[i + 1];
+            v[i] = a0 * cs.x - a1 * cs.y;
+            v[i + 1] = a0 * cs.y + a1 * cs.x;
+          }
+        }
+      }
+    }
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) store8(dst + c * 32 + i, v + i);
+    }
+  }
+}
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                      const __grid_constant__ CUtensorMap tB2, void* __restrict__ Y, int ldy,
-                     const __nv_bfloat16* R, int ldr, int M, int N, int K, int vec_ok, const GdnEpi ep) {
+                     const __nv_bfloat16* R, int ldr, int M, int N, int K, int vec_ok, const GdnEpi ep,
+                     const FaEpi fe) {
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;   // output columns per pair tile
   extern __shared__ uint8_t smem_raw[];
   // the same offsets in both CTAs: descriptors and barriers are addressed by offset
@@ -259,8 +328,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int row = m0 + (int)rank * BM + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       if (EPI == EPI_GDN) gdn_epilogue(t_row, row, n0, M, ep);
+      if (EPI == EPI_FA) fa_epilogue(t_row, row, n0, M, fe);
 #pragma unroll 1
-      for (int c = 0; c < (EPI == EPI_GDN ? 0 : OUT_COLS / 32); ++c) {
+      for (int c = 0; c < ((EPI == EPI_GDN || EPI == EPI_FA) ? 0 : OUT_COLS / 32); ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
         float v[32];
@@ -331,7 +401,8 @@ done:
 
 template <int EPI>
 static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2, const void* R, int ldr, void* Y,
-                          int ldy, int M, int N, int K, cudaStream_t s, const GdnEpi& ep = GdnEpi{}) {
+                          int ldy, int M, int N, int K, cudaStream_t s, const GdnEpi& ep = GdnEpi{},
+                          const FaEpi& fe = FaEpi{}) {
   constexpr int OUT_COLS = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   CUtensorMap tA, tB, tB2;
   if (!make_map(&tA, X, M, K, ldx, BM)) return cudaErrorNotSupported;
@@ -352,7 +423,7 @@ static cudaError_t launch(const void* X, int ldx, const void* W, const void* W2,
   const int vec_ok = ((ldy * esz) % 16 == 0) && (((uintptr_t)Y) % 16 == 0) &&
                      (EPI != EPI_ADD || ((ldr * 2) % 16 == 0 && ((uintptr_t)R) % 16 == 0));
   kern<<<(unsigned)(2 * pairs), 192, SMEM, s>>>(tA, tB, tB2, Y, ldy, (const __nv_bfloat16*)R, ldr, M, N, K, vec_ok,
-                                                 ep);
+                                                 ep, fe);
   return cudaGetLastError();
 }
 
@@ -377,6 +448,16 @@ cudaError_t linear_gdn(const void* X, int ldx, const void* W, int M, int K, cons
     return cudaErrorNotSupported;
   const int N = 3 * ep.H * 128 + 2 * ep.H;
   return tc::p2::launch<EPI_GDN>(X, ldx, W, nullptr, nullptr, 0, nullptr, 0, M, N, K, s, ep);
+}
+
+cudaError_t linear_fa(const void* X, int ldx, const void* W, int M, int K, const FaEpi& fe, cudaStream_t s) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+  if (M <= 128 || fe.T <= 0 || fe.rot < 0 || fe.rot > 64 || fe.rot % 2 || (fe.rot > 0 && !fe.rope) || !al16(X) ||
+      !al16(W) || (ldx * 2) % 16 || (K * 2) % 16 || !al16(fe.q) || !al16(fe.gate) || (fe.ld_gate * 2) % 16 ||
+      !al16(fe.k_slab) || !al16(fe.v_slab) || !al16(fe.q_gain) || !al16(fe.k_gain))
+    return cudaErrorNotSupported;
+  const int N = (2 * fe.Hq + 2 * fe.Hkv) * 256;
+  return tc::p2::launch<EPI_FA>(X, ldx, W, nullptr, nullptr, 0, nullptr, 0, M, N, K, s, GdnEpi{}, fe);
 }
 
 }  // namespace lk

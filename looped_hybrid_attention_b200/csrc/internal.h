@@ -7,7 +7,7 @@
 namespace lk {
 
 enum Dtype { F32 = 0, BF16 = 1 };
-enum Epilogue { EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_F32 = 3, EPI_GDN = 4 };
+enum Epilogue { EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_F32 = 3, EPI_GDN = 4, EPI_FA = 5 };
 
 // Outputs of the GDN input projection's fused epilogue (EPI_GDN): q, k L2-normalised per head,
 // v, and the gates g = -softplus(a + a_bias), beta = sigmoid(b + b_bias), from the columns
@@ -22,6 +22,28 @@ struct GdnEpi {
 // The projection with the GDN preparation in its epilogue (bf16, M > 128, dk = dv = 128,
 // H even); cudaErrorNotSupported otherwise.
 cudaError_t linear_gdn(const void* X, int ldx, const void* W, int M, int K, const GdnEpi& ep, cudaStream_t s);
+
+// Outputs of the FA input projection's fused epilogue (EPI_FA), from the columns
+// q | gate | k | v of the product (head dim 256): each q and k head RMS-normalised over its
+// 256 dims (eps inside the root), scaled by its gain and rotated on dims [0, rot) in
+// adjacent pairs by the position's (cos, sin) -- what fa_prep computes; q goes to a compact
+// buffer, k and v straight into the execution's slabs at their positions, the gate block
+// to its place in `gate` (row stride ld_gate).
+struct FaEpi {
+  void* q;                       // [M, Hq, 256] bf16
+  void* gate;                    // gate block of row m at gate + m * ld_gate
+  int ld_gate;
+  void *k_slab, *v_slab;         // [B, Hkv, kv_cap, 256] bf16
+  int kv_cap;
+  const void *q_gain, *k_gain;   // [256] bf16
+  float eps;
+  int Hq, Hkv, rot;              // rot <= 64
+  const float2* rope;            // [T, rot / 2] (cos, sin) of positions pos0 .. pos0 + T - 1
+  int T, pos0;                   // tokens per sequence (row m = b * T + t), position of t = 0
+};
+// The FA input projection with QK-norm, rotary and the KV write in its epilogue (bf16,
+// M > 128, head dim 256); cudaErrorNotSupported otherwise.
+cudaError_t linear_fa(const void* X, int ldx, const void* W, int M, int K, const FaEpi& fe, cudaStream_t s);
 enum MhcMode { MHC_OPEN = 0, MHC_MIX = 1, MHC_ROUTE = 2, MHC_MERGE = 3 };
 
 // ldx: row stride of x in elements (0 = d); r, sum_out and y are dense [M, d].

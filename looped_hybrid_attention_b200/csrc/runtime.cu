@@ -248,22 +248,37 @@ static loop_status run_layer(loop_model* m, loop_cache* c, const ExecRow& r, con
        "GDN output projection");
   } else {
     const int Hq = cf.fa_q_heads, Hkv = cf.fa_kv_heads, dh = cf.fa_head_dim;
-    gemm_work(M, m->in_fa, d, EPI_STORE, m->esize, fl, by);
-    CK(prof(m, s, P_GEMM, 1, fl, by,
-            [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d,
-                                EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
-       "FA input projection");
     char* kbase = (char*)c->kv.p + (size_t)r.slot * 2 * c->kv_slab_elems * m->esize;
     char* vbase = kbase + c->kv_slab_elems * m->esize;
-    // multi-token bf16 queries go raw to the tensor-core attention kernel, which applies
-    // their QK-norm and rotary as it stages them; the prep kernel then writes K and V only
-    const bool fuse_q = dt == BF16 && dh == 256 && T >= 16 && 128 % (Hq / Hkv) == 0 && cf.rotary_dims <= dh / 2;
-    CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * ((fuse_q ? 0 : Hq) + 2 * Hkv) * dh),
-            [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, fuse_q ? nullptr : m->gq.p, kbase, vbase,
-                                     c->max_tokens, B, T, pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base, cf.eps, dt,
-                                     s, (const float2*)m->rope.p); }),
-       "QK-norm / rotary / KV write");
     const char* gate = (const char*)m->proj.p + (size_t)Hq * dh * m->esize;
+    // prefill-sized bf16 batches: QK-norm, rotary and the KV write run in the projection's
+    // epilogue (normed, rotated q to a compact buffer; k, v into the slab; the gate block to
+    // its place in the projection buffer), so neither a preparation kernel nor a pass over
+    // the queries remains
+    auto al16 = [](const void* p) { return ((uintptr_t)p % 16) == 0; };
+    const bool fused_fa = dt == BF16 && M > 128 && dh == 256 && cf.rotary_dims <= 64 && al16(w.w_in) &&
+                          al16(w.q_norm) && al16(w.k_norm);
+    // otherwise multi-token bf16 queries go raw to the tensor-core attention kernel, which
+    // applies their QK-norm and rotary as it stages them; the prep kernel then writes K and V
+    const bool fuse_q = !fused_fa && dt == BF16 && dh == 256 && T >= 16 && 128 % (Hq / Hkv) == 0 &&
+                        cf.rotary_dims <= dh / 2;
+    gemm_work(M, m->in_fa, d, EPI_STORE, m->esize, fl, by);
+    if (fused_fa) {
+      const FaEpi fe{m->gq.p, (void*)gate, m->in_fa, kbase, vbase, c->max_tokens, w.q_norm, w.k_norm, cf.eps, Hq, Hkv,
+                     cf.rotary_dims, (const float2*)m->rope.p, T, pos0};
+      CK(prof(m, s, P_GEMM, 1, fl, by, [&] { return linear_fa(m->xn.p, d, w.w_in, (int)M, d, fe, s); }),
+         "FA input projection + QK-norm / rotary / KV write");
+    } else {
+      CK(prof(m, s, P_GEMM, 1, fl, by,
+              [&] { return linear(m->xn.p, d, w.w_in, nullptr, nullptr, 0, m->proj.p, m->in_fa, (int)M, m->in_fa, d,
+                                  EPI_STORE, dt, s, m->gemm_ws.p, m->gemm_ws.bytes); }),
+         "FA input projection");
+      CK(prof(m, s, P_FA_PREP, 1, 0, (double)M * es * (2.0 * ((fuse_q ? 0 : Hq) + 2 * Hkv) * dh),
+              [&] { return lk::fa_prep(m->proj.p, m->in_fa, w.q_norm, w.k_norm, fuse_q ? nullptr : m->gq.p, kbase,
+                                       vbase, c->max_tokens, B, T, pos0, Hq, Hkv, dh, cf.rotary_dims, cf.rope_base,
+                                       cf.eps, dt, s, (const float2*)m->rope.p); }),
+         "QK-norm / rotary / KV write");
+    }
     // causal (query, key) pairs: sum over new tokens of (pos0 + t + 1)
     const double pairs = (double)B * ((double)T * pos0 + (double)T * (T + 1) / 2.0);
     const double attn_bytes = es * ((double)M * Hq * dh * 3.0 + (double)B * Hkv * (pos0 + T) * dh * 2.0);
